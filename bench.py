@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""SPLA decode benchmark on B200: queries*heads/s and achieved HBM bandwidth.
+
+One step = the whole hot path for one batch: spla_append_kv (one new token
+per sequence, updating block statistics and the linear-attention state) then
+spla_decode (score every block -> select top-k -> exact attention over the
+kept blocks with the fused residual-linear-attention term -> combine).
+
+Default workload: batch 4, 32 query / 8 KV heads, d 128, 131072-token
+contexts in 64-token blocks, top-k 32, 64 steps of append + decode (the
+128K-context decode workload). Inputs are synthetic and seeded
+(workloads/gen.py) and resident in HBM before timing; L2 is flushed (a
+512 MiB write) before every timed step and the flush is outside the events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg3]
+    python bench.py --impl reference      # the CPU oracle on the host cores
+
+Multi-GPU (torchrun, one rank per GPU): every rank decodes its own
+independent batch (weak scaling, no collective on the data path); the step
+time is the max over ranks.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SPLA decode queries*heads/s (1 x B200), achieved HBM GB/s"
+UNIT = "queries*heads/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="cfg3")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (200 ms period)."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- bytes
+def step_bytes(w, sel: np.ndarray, lens: np.ndarray) -> dict:
+    """Algorithmic bytes of one decode: union of kept KV per (seq, KV head), all block
+    statistics, the S/z/m state (the count the target names), split by kernel."""
+    G = w.group
+    esz = 2 if w.dtype == "bf16" else 4
+    kv = stats = state = 0
+    for b in range(w.batch):
+        nb = -(-int(lens[b]) // w.block_size)
+        for h in range(w.num_kv_heads):
+            u = np.unique(sel[b, h * G:(h + 1) * G])
+            u = u[u >= 0]
+            for j in u:
+                n = min(w.block_size, int(lens[b]) - int(j) * w.block_size)
+                kv += 2 * n * w.head_dim * esz
+            stats += nb * 2 * w.head_dim * 4
+            state += (w.head_dim * w.head_dim + 2 * w.head_dim) * 4
+    return {"kv": kv, "stats": stats, "state": state, "total": kv + stats + state}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_linear_b200 import _lib
+    from workloads import feed_gpu, gen
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    w = gen.get(args.workload)
+    K, W = args.steps, args.warmup
+    cache = feed_gpu.build_cache(w, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    steps = [feed_gpu.step_inputs(w, s, device=dev) for s in range(W + 2 * K)]
+    gamma = torch.ones((w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    out = torch.empty((w.batch, w.num_q_heads, w.head_dim), dtype=steps[0][2].dtype, device=dev)
+    sels = torch.empty((2 * K, w.batch, w.num_q_heads, w.top_k + w.n_sink + w.n_local),
+                       dtype=torch.int32, device=dev)
+    lens_after = []
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+
+    def step(s, sel=None):
+        k, v, q = steps[s]
+        cache.append(k, v)
+        cache.decode(q, gamma, out, sel)
+
+    for s in range(W):
+        step(s)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    # ---- pass A: whole-step time (the value)
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    lens0 = cache.context_lens.cpu().numpy().copy()
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        for i in range(K):
+            flush.zero_()
+            ev0[i].record(stream)
+            step(W + i, sels[i])
+            ev1[i].record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    t_steps = [ev0[i].elapsed_time(ev1[i]) for i in range(K)]
+    t_total = sum(t_steps)
+
+    # ---- pass B: per-kernel events inside spla_decode (dominant-kernel roofline)
+    pe = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for row in pe:
+        for e in row:
+            e.record(stream)                  # materialise the handles
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        _lib.spla_profile_events([e.cuda_event for e in pe[i]])
+        step(W + K + i, sels[K + i])
+    _lib.spla_profile_events([])
+    torch.cuda.synchronize(dev)
+    kt = np.array([[pe[i][j].elapsed_time(pe[i][j + 1]) for j in range(4)] for i in range(K)])
+    kernel_names = ["score", "select", "decode", "combine"]
+
+    # ---- algorithmic bytes from the selections actually made
+    sel_np = sels.cpu().numpy()
+    lens_np = lens0 + 1 + np.arange(K)[:, None]          # each step appends one token first
+    by = [step_bytes(w, sel_np[i], lens_np[i]) for i in range(K)]
+    lens_b = lens0 + K + 1 + np.arange(K)[:, None]
+    byB = [step_bytes(w, sel_np[K + i], lens_b[i]) for i in range(K)]
+    status = cache.status()
+
+    # ---- e2e: host buffers through the same calls, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_pass(w, cache, steps, W + 2 * K, K, gamma, flush, dev, stream)
+
+    # ---- reduce over ranks
+    t_max = t_total
+    if world > 1:
+        tt = torch.tensor([t_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+        if e2e is not None:
+            te = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+            e2e["ms"] = float(te.item())
+    units_per_step = w.batch * w.num_q_heads
+    value = world * units_per_step * K / (t_max / 1e3)
+
+    if rank == 0:
+        hbm, peak_kind = peaks()
+        dec = kt[:, 2]
+        sco = kt[:, 0]
+        share = kt.sum(axis=0) / kt.sum()
+        dom = int(np.argmax(share))
+        dec_bytes = np.mean([b["kv"] + b["state"] for b in byB])
+        sco_bytes = np.mean([b["stats"] for b in byB])
+        dom_bytes = dec_bytes if dom == 2 else sco_bytes
+        dom_ms = float(np.mean(kt[:, dom]))
+        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+        step_gbs = np.mean([b["total"] for b in by]) / (t_total / K / 1e3) / 1e9
+        res = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": round(t_max / K, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded, workloads/gen.py)",
+            "config": {"workload": gen.DESCRIPTIONS[w.name], "name": w.name, "batch": w.batch,
+                       "context": int(w.context_lens[0]), "q_heads": w.num_q_heads,
+                       "kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                       "block": w.block_size, "top_k": w.top_k,
+                       "step": "spla_append_kv (1 token/seq) + spla_decode",
+                       "l2": "flushed (512 MiB write) before every timed step, outside the events",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "kernel": kernel_names[dom],
+                         "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(achieved / hbm, 4), "traffic": None,
+                         "peak_kind": f"{peak_kind} hbm_gbs",
+                         "bytes_per_launch": int(dom_bytes), "ms_per_launch": round(dom_ms, 5)},
+            "step_hbm": {"bytes_per_step": int(np.mean([b["total"] for b in by])),
+                         "kv_bytes": int(np.mean([b["kv"] for b in by])),
+                         "stats_bytes": int(np.mean([b["stats"] for b in by])),
+                         "state_bytes": int(np.mean([b["state"] for b in by])),
+                         "achieved_gbs": round(step_gbs, 1),
+                         "frac_of_peak": round(step_gbs / hbm, 4)},
+            "kernels_ms": {n: round(float(np.mean(kt[:, j])), 5) for j, n in enumerate(kernel_names)},
+            "kernel_share": {n: round(float(share[j]), 4) for j, n in enumerate(kernel_names)},
+            "clocks": clk.summary(),
+            "gpu_launches": 7 * K,
+            "dev_status": status,
+        }
+        if e2e is not None:
+            res["e2e"] = {"value": round(world * units_per_step * K / (e2e["ms"] / 1e3), 1),
+                          "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
+                          "d2h_bytes_per_step": e2e["d2h"]}
+        if not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_pass(w, cache, steps, s0, K, gamma, flush, dev, stream):
+    """Per step: pinned host -> device copy of (k, v, q), append + decode, device -> host of out."""
+    import torch
+    from workloads import gen
+    dt = steps[0][2].dtype
+    host = []
+    for i in range(K):
+        k, v = gen.step_tokens(w, s0 + i)
+        q = gen.query(w, s0 + i)
+        host.append(tuple(torch.from_numpy(a).to(dt).pin_memory() for a in (k[:, None], v[:, None], q)))
+    dk = torch.empty_like(steps[0][0])
+    dv = torch.empty_like(steps[0][1])
+    dq = torch.empty_like(steps[0][2])
+    out = torch.empty_like(dq)
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        e0[i].record(stream)
+        hk, hv, hq = host[i]
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        cache.append(dk, dv)
+        cache.decode(dq, gamma, out)
+        hout.copy_(out, non_blocking=True)
+        e1[i].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(e0[i].elapsed_time(e1[i]) for i in range(K))
+    h2d = sum(t.numel() * t.element_size() for t in host[0])
+    return {"ms": ms, "h2d": h2d, "d2h": hout.numel() * hout.element_size()}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, budget_s: float, steps: int = None):
+    """Time the oracle's decode (score, select, exact attention, RLA, combine) plus its
+    one-token append, on one (sequence, KV head) group of the workload: the G query
+    heads of that group are the units. Returns (units/s, units, seconds, description)."""
+    from oracle import feed as ofeed
+    from workloads import gen
+    oc = ofeed.build(w, groups=[(0, 0)])
+    gamma = gen.gamma(w)
+    units, t_spent, n = 0, 0.0, 0
+    while (steps is None and t_spent < budget_s) or (steps is not None and n < steps):
+        k, v = gen.step_tokens(w, n)
+        q = gen.query(w, n)
+        t0 = time.perf_counter()
+        oc.append_group(0, 0, k[0, 0][None], v[0, 0][None])
+        oc.decode(q, gamma)
+        t_spent += time.perf_counter() - t0
+        units += w.group
+        n += 1
+    desc = (f"oracle append(1 token) + decode of sequence 0, KV head 0 ({w.group} query heads) "
+            f"of the workload, {n} steps, {t_spent:.1f} s")
+    return units / t_spent, units, t_spent, desc, n
+
+
+def cpu_baseline(w):
+    v, units, secs, desc, n = oracle_sample(w, budget_s=12.0)
+    return {"value": round(v, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": desc}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from workloads import gen
+    w = gen.get(args.workload)
+    oracle_sample(w, 0.0, steps=args.warmup)                  # warm-up (untimed)
+    v, units, secs, desc, n = oracle_sample(w, 0.0, steps=args.steps)
+    res = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT,
+           "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(secs / n * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded, workloads/gen.py)",
+           "config": {"workload": gen.DESCRIPTIONS[w.name], "name": w.name},
+           "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": _threads(),
+                            "kind": "oracle", "sample": desc},
+           "e2e": {"value": round(v, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,285 @@
+// Host side of the C ABI declared in include/spla.h: argument checks,
+// workspace layout, TMA descriptors and the launch sequence.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace spla {
+cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s);
+cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, const void* v_new,
+                          const int32_t* n_new, int32_t max_new, int32_t* status, cudaStream_t s);
+cudaError_t launch_score(const CacheView& c, int dtype, const void* q, double scale,
+                         int first_order, float* scores, int chunk, int32_t* status,
+                         cudaStream_t s);
+cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
+                          const float* scores, uint32_t* bits, int nw, int32_t* nsel,
+                          int32_t* sel_idx, int kcap, cudaStream_t s);
+cudaError_t launch_decode_mma(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const void* q, float sl2, const uint32_t* bits, int nw, float* part,
+                              int nsplit, int max_per, int32_t* status, cudaStream_t s);
+cudaError_t launch_decode_simt(const CacheView& c, int dtype, const void* q, float sl2,
+                               const uint32_t* bits, int nw, float* part, int nsplit, int max_per,
+                               int32_t* status, cudaStream_t s);
+cudaError_t launch_combine(const CacheView& c, int dtype, const float* part, int nsplit,
+                           const int32_t* nsel, const float* gamma, float eps, int no_rla,
+                           void* out, float* o_sp, float* o_rl, cudaStream_t s);
+size_t mma_smem_for(int d, int bs, int max_per);
+size_t simt_smem_for(int d, int bs, int max_per);
+
+// The split heuristic is tuned for the 148-SM B200; results do not depend on it.
+constexpr int kTargetCtas = 148;
+constexpr int kMaxSmem = 227 * 1024;
+
+static thread_local int32_t g_last_cuda_error = 0;
+static thread_local cudaEvent_t g_prof[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+static thread_local bool g_prof_on = false;
+
+static void prof_mark(int i, cudaStream_t s) {
+    if (g_prof_on) cudaEventRecord(g_prof[i], s);
+}
+
+static spla_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = (int32_t)e;
+    return SPLA_ERR_CUDA;
+}
+
+static spla_status check_params(const spla_params* p) {
+    if (!p) return SPLA_ERR_INVALID_ARG;
+    if (p->num_q_heads <= 0 || p->num_kv_heads <= 0 || p->num_q_heads % p->num_kv_heads)
+        return SPLA_ERR_INVALID_ARG;
+    const int G = p->num_q_heads / p->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4) return SPLA_ERR_UNSUPPORTED;
+    if (p->head_dim != 64 && p->head_dim != 128) return SPLA_ERR_UNSUPPORTED;
+    if (p->block_size != 64 && p->block_size != 128) return SPLA_ERR_UNSUPPORTED;
+    if (p->top_k < 1 || p->n_sink < 0 || p->n_local < 0) return SPLA_ERR_INVALID_ARG;
+    if (p->dtype != SPLA_F32 && p->dtype != SPLA_BF16) return SPLA_ERR_UNSUPPORTED;
+    if (p->flags & ~(SPLA_FLAG_NO_RLA | SPLA_FLAG_FIRST_ORDER)) return SPLA_ERR_INVALID_ARG;
+    return SPLA_OK;
+}
+
+static spla_status check_cache(const spla_cache* c) {
+    if (!c) return SPLA_ERR_INVALID_ARG;
+    if (!c->k_pool || !c->v_pool || !c->blk_stats || !c->S || !c->z || !c->m ||
+        !c->block_table || !c->context_lens)
+        return SPLA_ERR_INVALID_ARG;
+    if (c->batch <= 0 || c->max_blocks_per_seq <= 0 || c->num_phys_blocks <= 0)
+        return SPLA_ERR_INVALID_ARG;
+    if (c->max_blocks_per_seq > SPLA_MAX_BLOCKS_PER_SEQ) return SPLA_ERR_CAPACITY;
+    return SPLA_OK;
+}
+
+static CacheView view_of(const spla_params* p, const spla_cache* c) {
+    CacheView v;
+    v.k_pool = c->k_pool;
+    v.v_pool = c->v_pool;
+    v.stats = c->blk_stats;
+    v.S = c->S;
+    v.z = c->z;
+    v.m = c->m;
+    v.table = c->block_table;
+    v.lens = c->context_lens;
+    v.batch = c->batch;
+    v.mbp = c->max_blocks_per_seq;
+    v.num_phys = c->num_phys_blocks;
+    v.hq = p->num_q_heads;
+    v.hkv = p->num_kv_heads;
+    v.group = p->num_q_heads / p->num_kv_heads;
+    v.d = p->head_dim;
+    v.bs = p->block_size;
+    return v;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) {
+    DecodeLayout L;
+    const int G = p->num_q_heads / p->num_kv_heads;
+    const int groups = batch * p->num_kv_heads;
+    L.kcap = p->top_k + p->n_sink + p->n_local;
+    L.nw = (mbp + 31) / 32;
+    L.rec = rec_floats(p->head_dim);
+    const int umax = (int)std::min<int64_t>(mbp, (int64_t)G * L.kcap);
+    int ns = (kTargetCtas + groups - 1) / groups;       // enough CTAs to cover the SMs once
+    ns = std::max(1, std::min(ns, std::max(1, umax / 2)));
+    L.nsplit = ns;
+    L.max_per = (umax + ns - 1) / ns + 1;
+    // scoring chunk: enough CTAs to fill the machine twice over
+    int chunk = 256;
+    while (chunk > 64 && (int64_t)groups * ((mbp + chunk - 1) / chunk) < 2 * kTargetCtas) chunk >>= 1;
+    L.score_chunk = chunk;
+    size_t off = 0;
+    L.off_scores = off;
+    off = align256(off + (size_t)batch * p->num_q_heads * mbp * sizeof(float));
+    L.off_bits = off;
+    off = align256(off + (size_t)batch * p->num_q_heads * L.nw * sizeof(uint32_t));
+    L.off_nsel = off;
+    off = align256(off + (size_t)batch * p->num_q_heads * sizeof(int32_t));
+    L.off_part = off;
+    off = align256(off + (size_t)groups * ns * G * L.rec * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D view of a pool as [num_phys*Hkv*B rows][d cols] bf16; box = B rows x 64 cols, 128B swizzle.
+static bool make_pool_map(CUtensorMap* m, const void* pool, const CacheView& c) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t rows = (cuuint64_t)c.num_phys * c.hkv * c.bs;
+    cuuint64_t dims[2] = {(cuuint64_t)c.d, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)c.d * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)c.bs};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace spla
+
+using namespace spla;
+
+extern "C" {
+
+int32_t spla_version(void) { return 100; }
+
+const char* spla_status_string(spla_status s) {
+    switch (s) {
+        case SPLA_OK: return "ok";
+        case SPLA_ERR_INVALID_ARG: return "invalid argument";
+        case SPLA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case SPLA_ERR_WORKSPACE: return "workspace missing or too small";
+        case SPLA_ERR_CAPACITY: return "size beyond a fixed limit";
+        case SPLA_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+int32_t spla_last_cuda_error(void) { return g_last_cuda_error; }
+
+spla_status spla_profile_events(void* const* events, int32_t n) {
+    if (n == 0) {
+        g_prof_on = false;
+        return SPLA_OK;
+    }
+    if (n != 5 || !events) return SPLA_ERR_INVALID_ARG;
+    for (int i = 0; i < 5; ++i) {
+        if (!events[i]) return SPLA_ERR_INVALID_ARG;
+        g_prof[i] = (cudaEvent_t)events[i];
+    }
+    g_prof_on = true;
+    return SPLA_OK;
+}
+
+spla_status spla_cache_init(const spla_params* params, const spla_cache* cache, void* stream) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if ((st = check_cache(cache)) != SPLA_OK) return st;
+    const CacheView v = view_of(params, cache);
+    cudaError_t e = launch_cache_init(v, (cudaStream_t)stream);
+    return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
+}
+
+spla_status spla_append_kv(const spla_params* params, const spla_cache* cache, const void* k_new,
+                           const void* v_new, const int32_t* n_new, int32_t max_new,
+                           int32_t* dev_status, void* stream) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if ((st = check_cache(cache)) != SPLA_OK) return st;
+    if (max_new < 0 || !n_new) return SPLA_ERR_INVALID_ARG;
+    if (max_new > 0 && (!k_new || !v_new)) return SPLA_ERR_INVALID_ARG;
+    if ((int64_t)max_new > (int64_t)cache->max_blocks_per_seq * params->block_size)
+        return SPLA_ERR_CAPACITY;
+    const CacheView v = view_of(params, cache);
+    cudaError_t e = launch_append(v, params->dtype, k_new, v_new, n_new, max_new, dev_status,
+                                  (cudaStream_t)stream);
+    return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
+}
+
+spla_status spla_decode_workspace_size(const spla_params* params, int32_t batch,
+                                       int32_t max_blocks_per_seq, size_t* bytes) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if (!bytes || batch <= 0 || max_blocks_per_seq <= 0) return SPLA_ERR_INVALID_ARG;
+    if (max_blocks_per_seq > SPLA_MAX_BLOCKS_PER_SEQ) return SPLA_ERR_CAPACITY;
+    *bytes = layout_of(params, batch, max_blocks_per_seq).total;
+    return SPLA_OK;
+}
+
+spla_status spla_decode(const spla_params* params, const spla_cache* cache, const void* q,
+                        const float* rms_gamma, void* out, int32_t* sel_idx, float* o_sparse_dbg,
+                        float* o_rla_dbg, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, void* stream) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if ((st = check_cache(cache)) != SPLA_OK) return st;
+    if (!q || !out) return SPLA_ERR_INVALID_ARG;
+    const DecodeLayout L = layout_of(params, cache->batch, cache->max_blocks_per_seq);
+    if (!workspace || workspace_bytes < L.total) return SPLA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return SPLA_ERR_WORKSPACE;
+    const CacheView v = view_of(params, cache);
+    const bool use_mma = params->dtype == SPLA_BF16;
+    const size_t smem = use_mma ? mma_smem_for(v.d, v.bs, L.max_per)
+                                : simt_smem_for(v.d, v.bs, L.max_per);
+    if (smem > (size_t)kMaxSmem) return SPLA_ERR_CAPACITY;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = static_cast<char*>(workspace);
+    float* scores = reinterpret_cast<float*>(ws + L.off_scores);
+    uint32_t* bits = reinterpret_cast<uint32_t*>(ws + L.off_bits);
+    int32_t* nsel = reinterpret_cast<int32_t*>(ws + L.off_nsel);
+    float* part = reinterpret_cast<float*>(ws + L.off_part);
+    const double scale = params->softmax_scale > 0.f ? (double)params->softmax_scale
+                                                     : 1.0 / sqrt((double)params->head_dim);
+    const float sl2 = (float)(scale * 1.4426950408889634);
+    const float eps = params->rms_eps > 0.f ? params->rms_eps : 1e-6f;
+    const int first_order = (params->flags & SPLA_FLAG_FIRST_ORDER) ? 1 : 0;
+    const int no_rla = (params->flags & SPLA_FLAG_NO_RLA) ? 1 : 0;
+
+    prof_mark(0, s);
+    cudaError_t e = launch_score(v, params->dtype, q, scale, first_order, scores, L.score_chunk,
+                                 dev_status, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    prof_mark(1, s);
+    e = launch_select(v, params->top_k, params->n_sink, params->n_local, scores, bits, L.nw, nsel,
+                      sel_idx, L.kcap, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    prof_mark(2, s);
+    if (use_mma) {
+        CUtensorMap tk, tv;
+        if (!make_pool_map(&tk, v.k_pool, v) || !make_pool_map(&tv, v.v_pool, v))
+            return cuda_fail(cudaErrorInvalidValue);
+        e = launch_decode_mma(v, tk, tv, q, sl2, bits, L.nw, part, L.nsplit, L.max_per, dev_status,
+                              s);
+    } else {
+        e = launch_decode_simt(v, params->dtype, q, sl2, bits, L.nw, part, L.nsplit, L.max_per,
+                               dev_status, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    prof_mark(3, s);
+    e = launch_combine(v, params->dtype, part, L.nsplit, nsel, rms_gamma, eps, no_rla, out,
+                       o_sparse_dbg, o_rla_dbg, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    prof_mark(4, s);
+    return SPLA_OK;
+}
+
+}  // extern "C"

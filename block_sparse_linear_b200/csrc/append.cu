@@ -1,0 +1,197 @@
+// a0 -- appending tokens: write K/V into the paged pool, recompute the block
+// statistics of every touched block, and update the global linear-attention
+// state (SPLA technical summary, gist.science: section 2.1 for the per-block
+// mean and diagonal variance, section 2.2 for the global state that linear
+// attention over all blocks reads, section 2.3 for the feature map exp).
+//
+// Three launches, stream-ordered:
+//   append_kv_stats  grid (touched blocks, batch*Hkv): write tokens, then the
+//                    block's mean and population variance in fp64 (two-pass);
+//   append_state     grid (d/8 row groups, batch*Hkv): m <- max(m, k_new),
+//                    rescale S and z rows by exp(m_old - m_new), add
+//                    exp(k - m_new) v^T and exp(k - m_new);
+//   append_advance   one CTA: context_lens[b] += n_new[b].
+// The first two read the old context_lens and are independent of each other.
+#include "common.cuh"
+
+namespace spla {
+
+// Validation shared by the three kernels: the same answer in each.
+__device__ __forceinline__ bool append_ok(const CacheView& c, const int32_t* n_new,
+                                          int32_t max_new, int b, int32_t* L0, int32_t* n) {
+    int32_t l0 = c.lens[b];
+    int32_t nn = n_new[b];
+    *L0 = l0;
+    *n = nn;
+    if (nn < 0 || nn > max_new) return false;
+    if (l0 < 0 || (int64_t)l0 + nn > (int64_t)c.mbp * c.bs) return false;
+    return true;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) append_kv_stats_kernel(CacheView c, const T* k_new,
+                                                              const T* v_new,
+                                                              const int32_t* n_new,
+                                                              int32_t max_new, int32_t* status) {
+    const int b = blockIdx.y / c.hkv;
+    const int h = blockIdx.y % c.hkv;
+    int32_t L0, n;
+    if (!append_ok(c, n_new, max_new, b, &L0, &n)) {
+        if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0)
+            set_status(status, (n < 0 || n > max_new) ? SPLA_DEV_BAD_COUNT : SPLA_DEV_CAPACITY);
+        return;
+    }
+    if (n == 0) return;
+    const int bs = c.bs, d = c.d;
+    const int lb = L0 / bs + blockIdx.x;            // logical block this CTA owns
+    const int64_t blk_lo = (int64_t)lb * bs;
+    if (blk_lo >= (int64_t)L0 + n) return;
+    const int32_t phys = c.table[(int64_t)b * c.mbp + lb];
+    if (phys < 0 || phys >= c.num_phys) {
+        if (threadIdx.x == 0) set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
+        return;
+    }
+    const int t_beg = (int)(blk_lo > L0 ? blk_lo : (int64_t)L0);
+    const int t_end = (int)((int64_t)L0 + n < blk_lo + bs ? (int64_t)L0 + n : blk_lo + bs);
+    T* kp = (T*)c.k_pool + ((int64_t)phys * c.hkv + h) * bs * d;
+    T* vp = (T*)c.v_pool + ((int64_t)phys * c.hkv + h) * bs * d;
+    // write the new tokens of this block
+    const int nw = (t_end - t_beg) * d;
+    for (int e = threadIdx.x; e < nw; e += blockDim.x) {
+        const int t = t_beg + e / d, i = e % d;
+        const int64_t src = (((int64_t)b * max_new + (t - L0)) * c.hkv + h) * d + i;
+        kp[(int64_t)(t - blk_lo) * d + i] = k_new[src];
+        vp[(int64_t)(t - blk_lo) * d + i] = v_new[src];
+    }
+    __syncthreads();
+    // statistics over all tokens now in the block: two passes in fp64
+    const int nj = t_end - (int)blk_lo;
+    float* st = c.stats + ((int64_t)phys * c.hkv + h) * 2 * d;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+        double s = 0.0;
+        for (int t = 0; t < nj; ++t) s += (double)to_f(kp[(int64_t)t * d + i]);
+        const double mean = s / nj;
+        double q = 0.0;
+        for (int t = 0; t < nj; ++t) {
+            const double x = (double)to_f(kp[(int64_t)t * d + i]) - mean;
+            q += x * x;
+        }
+        st[i] = (float)mean;
+        st[d + i] = (float)(q / nj);
+    }
+}
+
+// Rows [8*blockIdx.x, +8) of S (and the same entries of z, m) of one (sequence, KV head).
+// Warp r owns row r; lane l owns columns l, l+32, ... of that row.
+template <typename T>
+__global__ void __launch_bounds__(256) append_state_kernel(CacheView c, const T* k_new,
+                                                           const T* v_new, const int32_t* n_new,
+                                                           int32_t max_new) {
+    const int b = blockIdx.y / c.hkv;
+    const int h = blockIdx.y % c.hkv;
+    int32_t L0, n;
+    if (!append_ok(c, n_new, max_new, b, &L0, &n) || n == 0) return;
+    const int d = c.d;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= d) return;
+    const int64_t gidx = ((int64_t)b * c.hkv + h) * d + row;
+    float* Srow = c.S + gidx * d;
+    auto kval = [&](int t) -> float {
+        return to_f(k_new[(((int64_t)b * max_new + t) * c.hkv + h) * d + row]);
+    };
+    // running max of this dimension over the new tokens
+    float mx = -SPLA_INF;
+    for (int t = lane; t < n; t += 32) mx = fmaxf(mx, kval(t));
+    mx = warp_max(mx);
+    const float m_old = c.m[gidx];
+    const float m_new = fmaxf(m_old, mx);
+    const float f = (m_old == -SPLA_INF) ? 0.f : expf(m_old - m_new);
+    constexpr int CPL = 4;                         // columns per lane (d <= 128)
+    float acc[CPL], tot[CPL];
+#pragma unroll
+    for (int u = 0; u < CPL; ++u) {
+        const int j = lane + 32 * u;
+        tot[u] = (j < d) ? Srow[j] * f : 0.f;
+        acc[u] = 0.f;
+    }
+    float zacc = 0.f, ztot = c.z[gidx] * f;
+    // new tokens, summed in chunks of 256 before joining the running total
+    for (int t = 0; t < n; ++t) {
+        const float e = expf(kval(t) - m_new);
+        const T* vr = v_new + (((int64_t)b * max_new + t) * c.hkv + h) * d;
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) {
+            const int j = lane + 32 * u;
+            if (j < d) acc[u] = fmaf(e, to_f(vr[j]), acc[u]);
+        }
+        zacc += e;
+        if ((t & 255) == 255) {
+#pragma unroll
+            for (int u = 0; u < CPL; ++u) { tot[u] += acc[u]; acc[u] = 0.f; }
+            ztot += zacc;
+            zacc = 0.f;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < CPL; ++u) {
+        const int j = lane + 32 * u;
+        if (j < d) Srow[j] = tot[u] + acc[u];
+    }
+    if (lane == 0) {
+        c.z[gidx] = ztot + zacc;
+        c.m[gidx] = m_new;
+    }
+}
+
+__global__ void append_advance_kernel(CacheView c, const int32_t* n_new, int32_t max_new) {
+    for (int b = threadIdx.x; b < c.batch; b += blockDim.x) {
+        int32_t L0, n;
+        if (append_ok(c, n_new, max_new, b, &L0, &n)) c.lens[b] = L0 + n;
+    }
+}
+
+__global__ void cache_init_kernel(CacheView c) {
+    const int64_t nsz = (int64_t)c.batch * c.hkv * c.d;
+    const int64_t ssz = nsz * c.d;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < ssz;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        c.S[i] = 0.f;
+        if (i < nsz) {
+            c.z[i] = 0.f;
+            c.m[i] = -SPLA_INF;
+        }
+        if (i < c.batch) c.lens[i] = 0;
+    }
+}
+
+// ------------------------------------------------------------------ host launchers
+cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s) {
+    cache_init_kernel<<<296, 256, 0, s>>>(c);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, const void* v_new,
+                          const int32_t* n_new, int32_t max_new, int32_t* status,
+                          cudaStream_t s) {
+    if (max_new > 0) {
+        dim3 g1((max_new + c.bs - 1) / c.bs + 1, c.batch * c.hkv);
+        dim3 g2((c.d + 7) / 8, c.batch * c.hkv);
+        if (dtype == SPLA_BF16) {
+            append_kv_stats_kernel<__nv_bfloat16><<<g1, 256, 0, s>>>(
+                c, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_new, max_new, status);
+            append_state_kernel<__nv_bfloat16><<<g2, 256, 0, s>>>(
+                c, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_new, max_new);
+        } else {
+            append_kv_stats_kernel<float><<<g1, 256, 0, s>>>(c, (const float*)k_new,
+                                                            (const float*)v_new, n_new, max_new,
+                                                            status);
+            append_state_kernel<float><<<g2, 256, 0, s>>>(c, (const float*)k_new,
+                                                         (const float*)v_new, n_new, max_new);
+        }
+    }
+    append_advance_kernel<<<1, 128, 0, s>>>(c, n_new, max_new);
+    return cudaGetLastError();
+}
+
+}  // namespace spla

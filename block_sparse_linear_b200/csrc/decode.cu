@@ -1,0 +1,786 @@
+// a3 + a4 + a5 -- split-KV decode over the kept blocks with the residual linear
+// attention computed in the same pass, then the split combine (SPLA technical
+// summary, gist.science: section 2 opening -- exact attention over the kept
+// blocks; section 2.2 -- RLA by subtraction, the kept blocks' linear-attention
+// term computed while they are on chip so unkept blocks are never read;
+// section 2.3 -- exponential feature map, RMS-normalised RLA added to the
+// sparse output). Softmax is softmax(q k^T / sqrt(d)) as in the Baidu article
+// "Sparse Attention for Long-Context LLMs: Implementation and Trade-off
+// Design", section 1; normalised linear attention as in its section 7.
+//
+// Grid (nsplit, batch*Hkv). Every CTA of a (sequence, KV head) group:
+//   * forms the union of the G heads' selections from their bitsets and takes
+//     an equal share of it (the union is read once for all G heads; a head
+//     that did not select a block is masked out of that block);
+//   * reads rows [s*d/nsplit, (s+1)*d/nsplit) of the state S, z and computes
+//     that slice of the global linear-attention readout N, D;
+//   * streams its blocks' K and V tiles and accumulates, per head, the online
+//     softmax (m, l, acc = sum p v) and the kept blocks' linear-attention
+//     numerator and denominator (N~ = sum w v, D~ = sum w) with
+//     w_t = sum_i exp(q_i + m_i - c) exp(k_t,i - m_i);
+//   * writes one partial record per head: m, l, acc, R = N_slice - N~, Dr = D_slice - D~.
+// combine_kernel merges the records of a head: the log-sum-exp merge of the
+// softmax partials, o_rla = sum R / sum Dr, RMSNorm, out = o_sparse + gamma*RMSNorm(o_rla).
+//
+// decode_mma_kernel (bf16 K/V): 4 consumer warps + 1 TMA producer warp. Each
+// (block, KV head) K or V tile is fetched by 2-D tiled TMA (128-byte swizzle,
+// no multicast) into a STAGES-deep mbarrier ring. Per 16-token slab a warp
+// runs the G-head contractions on tensor cores (mma.sync m16n8k16 bf16):
+//   logits  = K(16 x d) . Q^T(d x 8)            (q exact in bf16)
+//   w       = phi(K)(16 x d) . [a_hi a_lo]^T    (phi(K) split hi/lo in bf16)
+//   O^T    += V^T(d x 16) . [P W]_{hi,lo}       (P, W split hi/lo in bf16)
+// so every computed operand carries ~16 mantissa bits and sums are fp32.
+// decode_simt_kernel (fp32 or bf16 K/V): plain fp32 FMA, for the fp32 path.
+#include "common.cuh"
+
+namespace spla {
+
+// ------------------------------------------------------------------ shared prologue pieces
+// Union of the G heads' selections for this CTA's share (run by one warp).
+// Writes blk[], phys[], hm[] for union positions [u0, u1) and returns u1 - u0.
+__device__ int build_union_share(const CacheView& c, const uint32_t* bits, int nw, int b, int h,
+                                 int nb, int split, int nsplit, int max_per, int32_t* blk,
+                                 int32_t* phys, uint32_t* hm, int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int G = c.group;
+    const int nwu = (nb + 31) >> 5;
+    const int wpl = (nwu + 31) >> 5;
+    const uint32_t* hb = bits + ((int64_t)b * c.hq + h * G) * nw;
+    auto word = [&](int w) -> uint32_t {
+        uint32_t u = 0u;
+        for (int g = 0; g < G; ++g) u |= hb[(int64_t)g * nw + w];
+        if (w == nwu - 1 && (nb & 31)) u &= (1u << (nb & 31)) - 1u;
+        return u;
+    };
+    const int w0 = lane * wpl, w1 = min(nwu, w0 + wpl);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(word(w));
+    int x = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    const int U = __shfl_sync(0xffffffffu, x, 31);
+    const int u0 = (int)(((int64_t)split * U) / nsplit);
+    const int u1 = (int)(((int64_t)(split + 1) * U) / nsplit);
+    int r = x - cnt;
+    for (int w = w0; w < w1 && r < u1; ++w) {
+        uint32_t u = word(w);
+        const int pc = __popc(u);
+        if (r + pc <= u0) { r += pc; continue; }
+        while (u) {
+            const int bit = __ffs(u) - 1;
+            u &= u - 1u;
+            if (r >= u0 && r < u1) {
+                const int idx = r - u0;
+                const int j = (w << 5) + bit;
+                uint32_t mask = 0u;
+                for (int g = 0; g < G; ++g) mask |= ((hb[(int64_t)g * nw + w] >> bit) & 1u) << g;
+                int32_t p = c.table[(int64_t)b * c.mbp + j];
+                if (p < 0 || p >= c.num_phys) {
+                    set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
+                    p = 0;
+                    mask = 0u;
+                }
+                if (idx < max_per) {
+                    blk[idx] = j;
+                    phys[idx] = p;
+                    hm[idx] = mask;
+                }
+            }
+            ++r;
+        }
+    }
+    return min(u1 - u0, max_per);
+}
+
+// Query-side constants (run by nthr threads with barrier id `bar`):
+//   qs[g][i] = q (fp32), a[g][i] = exp(q_i + m_i - c_g), ml[i] = m_i*log2e.
+__device__ void query_setup(const CacheView& c, const void* q, int dtype, int b, int h,
+                            float* qs, float* a, float* ml, float* cg, int tid, int nthr) {
+    const int G = c.group, d = c.d;
+    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
+    for (int e = tid; e < G * d; e += nthr) {
+        const int g = e / d, i = e % d;
+        const int64_t qi = ((int64_t)b * c.hq + h * G + g) * d + i;
+        qs[e] = dtype == SPLA_BF16 ? __bfloat162float(((const __nv_bfloat16*)q)[qi])
+                                   : ((const float*)q)[qi];
+    }
+    for (int i = tid; i < d; i += nthr) ml[i] = mrow[i] * SPLA_LOG2E;
+}
+
+__device__ void query_weights(const CacheView& c, int b, int h, const float* qs, float* a,
+                              float* cg, int tid, int nthr) {
+    const int G = c.group, d = c.d;
+    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < G) {
+        float mx = -SPLA_INF;
+        for (int i = lane; i < d; i += 32) mx = fmaxf(mx, qs[warp * d + i] + mrow[i]);
+        mx = warp_max(mx);
+        if (lane == 0) cg[warp] = mx;
+    }
+}
+
+// ------------------------------------------------------------------ bf16 tensor-core kernel
+template <int D, int BS, int STAGES>
+struct MmaCfg {
+    static constexpr int NCW = 4;                           // consumer warps
+    static constexpr int THREADS = (NCW + 1) * 32;
+    static constexpr int BOXES = D / 64;                    // 64-column boxes per tile
+    static constexpr int BOX_BYTES = BS * 128;
+    static constexpr int TILE_BYTES = BOXES * BOX_BYTES;    // one of K or V
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+    static constexpr int SLABS = BS / 16;
+};
+
+template <int D, int BS, int STAGES>
+__global__ void __launch_bounds__(MmaCfg<D, BS, STAGES>::THREADS, 1)
+decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __nv_bfloat16* __restrict__ q,
+                  float sl2, const uint32_t* __restrict__ bits, int nw, float* __restrict__ part,
+                  int nsplit, int max_per, int32_t* status) {
+    using Cfg = MmaCfg<D, BS, STAGES>;
+    constexpr int NCW = Cfg::NCW, G4 = 4;
+    extern __shared__ __align__(1024) unsigned char smem_mma[];
+    // carve: stages (1024-aligned) | barriers | lists | query constants
+    unsigned char* base = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_mma) + 1023) & ~uintptr_t(1023));
+    unsigned char* stages = base;
+    uint64_t* full = reinterpret_cast<uint64_t*>(stages + STAGES * Cfg::STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    int32_t* blk = reinterpret_cast<int32_t*>(empty + STAGES);
+    int32_t* phys = blk + max_per;
+    uint32_t* hm = reinterpret_cast<uint32_t*>(phys + max_per);
+    float* qs = reinterpret_cast<float*>(hm + max_per);     // [4][D]
+    float* aw = qs + G4 * D;                                // [4][D]
+    float* ml = aw + G4 * D;                                // [D]
+    float* nsl = ml + D;                                    // [4][D]
+    float* dsl = nsl + G4 * D;                              // [4]
+    float* cg = dsl + G4;                                   // [4]
+    __shared__ int s_nblk, s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv, split = blockIdx.x;
+    const int G = c.group;
+    int32_t L = c.lens[b];
+    if (L < 0 || L > c.mbp * c.bs) L = max(0, min(L, c.mbp * c.bs));
+    const int nb = (L + BS - 1) / BS;
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NCW);
+        }
+        fence_barrier_init();
+        s_abort = 0;
+    }
+    if (warp == NCW) {
+        const int n = (nb > 0) ? build_union_share(c, bits, nw, b, h, nb, split, nsplit, max_per,
+                                                   blk, phys, hm, status)
+                               : 0;
+        if (lane == 0) s_nblk = n;
+    } else if (nb > 0) {
+        query_setup(c, q, SPLA_BF16, b, h, qs, aw, ml, cg, tid, NCW * 32);
+        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
+        query_weights(c, b, h, qs, aw, cg, tid, NCW * 32);
+        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
+        const float* mrow = c.m + ((int64_t)b * c.hkv + h) * D;
+        for (int e = tid; e < G * D; e += NCW * 32) {
+            const int g = e / D, i = e % D;
+            aw[e] = expf(qs[e] + mrow[i] - cg[g]);
+        }
+    }
+    __syncthreads();
+    const int nblk = s_nblk;
+    const int64_t rec_base = (((int64_t)b * c.hkv + h) * nsplit + split) * G;
+    const int REC = rec_floats(D);
+
+    if (nb == 0) {
+        for (int e = tid; e < G * REC; e += blockDim.x) {
+            const int g = e / REC, f = e % REC;
+            part[(rec_base + g) * REC + f] = (f == 0) ? -SPLA_INF : 0.f;
+        }
+        return;
+    }
+
+    // per-lane consumer state (columns c0, c1 of the C fragments; see below)
+    float m_run[2] = {-SPLA_INF, -SPLA_INF}, l_run[2] = {0.f, 0.f}, dt_run[2] = {0.f, 0.f};
+    float acc[D / 16][4];
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    const int c0 = 2 * (lane & 3), c1 = c0 + 1;
+
+    if (warp == NCW) {
+        // ---------------- producer: TMA ring
+        if (lane == 0) {
+            for (int it = 0; it < nblk; ++it) {
+                const int st = it % STAGES;
+                if (it >= STAGES) {
+                    if (!mbar_wait_bounded(&empty[st], ((it / STAGES) - 1) & 1)) {
+                        set_status(status, SPLA_DEV_TIMEOUT);
+                        atomicExch(&s_abort, 1);
+                        break;
+                    }
+                }
+                if (*(volatile int*)&s_abort) break;
+                unsigned char* kst = stages + st * Cfg::STAGE_BYTES;
+                unsigned char* vst = kst + Cfg::TILE_BYTES;
+                mbar_arrive_expect_tx(&full[st], Cfg::STAGE_BYTES);
+                const int row = (phys[it] * c.hkv + h) * BS;
+#pragma unroll
+                for (int bx = 0; bx < Cfg::BOXES; ++bx) {
+                    tma_load_2d(kst + bx * Cfg::BOX_BYTES, &tmK, &full[st], bx * 64, row);
+                    tma_load_2d(vst + bx * Cfg::BOX_BYTES, &tmV, &full[st], bx * 64, row);
+                }
+            }
+        }
+    } else {
+        // ---------------- consumers
+        // slice of the global readout: rows [r0, r1) of S and z
+        const int r0 = (int)((int64_t)split * D / nsplit), r1 = (int)((int64_t)(split + 1) * D / nsplit);
+        const float* Sg = c.S + ((int64_t)b * c.hkv + h) * D * D;
+        const float* zg = c.z + ((int64_t)b * c.hkv + h) * D;
+        for (int j = tid; j < D; j += NCW * 32) {
+            float acc[G4] = {0.f, 0.f, 0.f, 0.f};
+            for (int i = r0; i < r1; ++i) {
+                const float sv = Sg[(int64_t)i * D + j];
+#pragma unroll
+                for (int g = 0; g < G4; ++g)
+                    if (g < G) acc[g] = fmaf(aw[g * D + i], sv, acc[g]);
+            }
+#pragma unroll
+            for (int g = 0; g < G4; ++g)
+                if (g < G) nsl[g * D + j] = acc[g];
+        }
+        if (warp < G) {
+            float s = 0.f;
+            for (int i = r0 + lane; i < r1; i += 32) s = fmaf(aw[warp * D + i], zg[i], s);
+            s = warp_sum(s);
+            if (lane == 0) dsl[warp] = s;
+        }
+        // B fragments: column n = lane/4; rows k = 2*(lane%4) (+1, +8, +9) of each 16-dim step
+        uint32_t qf[D / 16][2], wf[D / 16][2];
+        {
+            const int n = lane >> 2;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int kb = kk * 16 + 2 * (lane & 3);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int i = kb + 8 * half;
+                    qf[kk][half] = (n < G) ? pack_bf16(qs[n * D + i], qs[n * D + i + 1]) : 0u;
+                    uint32_t wv = 0u;
+                    const int g = n & 3;
+                    if (g < G) {
+                        const float x0 = aw[g * D + i], x1 = aw[g * D + i + 1];
+                        const uint32_t hi = pack_bf16(x0, x1);
+                        wv = (n < 4) ? hi : pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
+                    }
+                    wf[kk][half] = wv;
+                }
+            }
+        }
+        const bool lo_half = (lane & 3) < 2;
+
+        for (int it = 0; it < nblk; ++it) {
+            const int st = it % STAGES;
+            if (!mbar_wait_bounded(&full[st], (it / STAGES) & 1)) {
+                set_status(status, SPLA_DEV_TIMEOUT);
+                atomicExch(&s_abort, 1);
+                break;
+            }
+            const unsigned char* kst = stages + st * Cfg::STAGE_BYTES;
+            unsigned char* vst = const_cast<unsigned char*>(kst) + Cfg::TILE_BYTES;
+            const int jblk = blk[it];
+            const int nvalid = min(BS, L - jblk * BS);
+            const uint32_t hmask = hm[it];
+            const uint32_t kbase = smem_u32(kst), vbase = smem_u32(vst);
+            if (hmask) {
+                for (int sl = warp; sl < Cfg::SLABS; sl += NCW) {
+                    const int t0 = sl * 16;
+                    if (t0 >= nvalid) break;
+                    if (t0 + 16 > nvalid) {
+                        // rows past the sequence end: zero V so that p = 0 rows add nothing
+                        for (int e = lane; e < 16 * (D / 8); e += 32) {
+                            const int r = t0 + e / (D / 8), ch = e % (D / 8);
+                            if (r >= nvalid)
+                                *reinterpret_cast<uint4*>(vst + (ch >> 3) * Cfg::BOX_BYTES +
+                                                          swz128(r, ch & 7)) = make_uint4(0, 0, 0, 0);
+                        }
+                        fence_proxy_async();
+                        __syncwarp();
+                    }
+                    float cl[4] = {0.f, 0.f, 0.f, 0.f}, cw1[4] = {0.f, 0.f, 0.f, 0.f},
+                          cw2[4] = {0.f, 0.f, 0.f, 0.f};
+                    const int qm = lane >> 3, rr = lane & 7;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const int t = t0 + rr + ((qm & 1) << 3);
+                        const int ch = ((kk & 3) << 1) + (qm >> 1);
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4(kbase + (kk >> 2) * Cfg::BOX_BYTES + swz128(t, ch), a0, a1, a2, a3);
+                        mma_bf16(cl, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                        const int kb = kk * 16 + 2 * (lane & 3);
+                        const float2 mA = *reinterpret_cast<const float2*>(ml + kb);
+                        const float2 mB = *reinterpret_cast<const float2*>(ml + kb + 8);
+                        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+                        auto phi = [&](uint32_t kr, float m0, float m1, uint32_t& hi, uint32_t& lo) {
+                            const float x0 = ex2(fmaf(bf16_lo(kr), SPLA_LOG2E, -m0));
+                            const float x1 = ex2(fmaf(bf16_hi(kr), SPLA_LOG2E, -m1));
+                            hi = pack_bf16(x0, x1);
+                            lo = pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
+                        };
+                        phi(a0, mA.x, mA.y, h0, l0);
+                        phi(a1, mA.x, mA.y, h1, l1);
+                        phi(a2, mB.x, mB.y, h2, l2);
+                        phi(a3, mB.x, mB.y, h3, l3);
+                        mma_bf16(cw1, h0, h1, h2, h3, wf[kk][0], wf[kk][1]);
+                        mma_bf16(cw2, l0, l1, l2, l3, wf[kk][0], wf[kk][1]);
+                    }
+                    // W = hi-part columns + lo-part columns (cols g and g+4)
+                    float x[4], y[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        x[r] = cw1[r] + cw2[r];
+                        y[r] = __shfl_down_sync(0xffffffffu, x[r], 2);
+                    }
+                    const int tr0 = t0 + (lane >> 2), tr1 = tr0 + 8;
+                    const bool hc0 = lo_half && c0 < G && ((hmask >> c0) & 1u);
+                    const bool hc1 = lo_half && c1 < G && ((hmask >> c1) & 1u);
+                    const bool v00 = hc0 && tr0 < nvalid, v01 = hc1 && tr0 < nvalid;
+                    const bool v10 = hc0 && tr1 < nvalid, v11 = hc1 && tr1 < nvalid;
+                    const float s00 = v00 ? cl[0] * sl2 : -SPLA_INF, s01 = v01 ? cl[1] * sl2 : -SPLA_INF;
+                    const float s10 = v10 ? cl[2] * sl2 : -SPLA_INF, s11 = v11 ? cl[3] * sl2 : -SPLA_INF;
+                    const float w00 = v00 ? x[0] + y[0] : 0.f, w01 = v01 ? x[1] + y[1] : 0.f;
+                    const float w10 = v10 ? x[2] + y[2] : 0.f, w11 = v11 ? x[3] + y[3] : 0.f;
+                    float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+                    }
+                    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+                    const float f0 = (mn0 == -SPLA_INF) ? 1.f : ex2(m_run[0] - mn0);
+                    const float f1 = (mn1 == -SPLA_INF) ? 1.f : ex2(m_run[1] - mn1);
+                    const float p00 = v00 ? ex2(s00 - mn0) : 0.f, p10 = v10 ? ex2(s10 - mn0) : 0.f;
+                    const float p01 = v01 ? ex2(s01 - mn1) : 0.f, p11 = v11 ? ex2(s11 - mn1) : 0.f;
+                    l_run[0] = l_run[0] * f0 + p00 + p10;
+                    l_run[1] = l_run[1] * f1 + p01 + p11;
+                    m_run[0] = mn0;
+                    m_run[1] = mn1;
+                    dt_run[0] += w00 + w10;
+                    dt_run[1] += w01 + w11;
+                    const float g0 = lo_half ? f0 : 1.f, g1 = lo_half ? f1 : 1.f;
+#pragma unroll
+                    for (int mt = 0; mt < D / 16; ++mt) {
+                        acc[mt][0] *= g0;
+                        acc[mt][1] *= g1;
+                        acc[mt][2] *= g0;
+                        acc[mt][3] *= g1;
+                    }
+                    // [P | W] as a 16 x 8 matrix in C layout: lanes with cols 4..7 take W from lane-2
+                    float wv[4] = {w00, w01, w10, w11}, pw[4];
+                    const float pv[4] = {p00, p01, p10, p11};
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const float up = __shfl_up_sync(0xffffffffu, wv[r], 2);
+                        pw[r] = lo_half ? pv[r] : up;
+                    }
+                    const uint32_t hA = pack_bf16(pw[0], pw[1]), hB = pack_bf16(pw[2], pw[3]);
+                    const uint32_t lA = pack_bf16(pw[0] - bf16_lo(hA), pw[1] - bf16_hi(hA));
+                    const uint32_t lB = pack_bf16(pw[2] - bf16_lo(hB), pw[3] - bf16_hi(hB));
+                    const uint32_t bh0 = movmatrix_t(hA), bh1 = movmatrix_t(hB);
+                    const uint32_t bl0 = movmatrix_t(lA), bl1 = movmatrix_t(lB);
+#pragma unroll
+                    for (int mt = 0; mt < D / 16; ++mt) {
+                        const int t = t0 + rr + ((qm >> 1) << 3);
+                        const int ch = ((mt & 3) << 1) + (qm & 1);
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4_t(vbase + (mt >> 2) * Cfg::BOX_BYTES + swz128(t, ch), a0, a1, a2, a3);
+                        mma_bf16(acc[mt], a0, a1, a2, a3, bh0, bh1);
+                        mma_bf16(acc[mt], a0, a1, a2, a3, bl0, bl1);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        // reduce the lane partials of l and D~ over the 8 lanes of each column
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                l_run[e] += __shfl_xor_sync(0xffffffffu, l_run[e], o);
+                dt_run[e] += __shfl_xor_sync(0xffffffffu, dt_run[e], o);
+            }
+    }
+    // every consumer is done with the stage buffers once all threads pass here
+    __syncthreads();
+    if (warp < NCW) {
+        // park per-warp results in the (now idle) stage buffers
+        float* mw = reinterpret_cast<float*>(stages);               // [NCW][4]
+        float* lw = mw + NCW * 4;
+        float* dw = lw + NCW * 4;
+        float* ap = dw + NCW * 4;                                   // [NCW][4][D]
+        float* an = ap + NCW * 4 * D;                               // [NCW][4][D]
+        if (lane < 2) {
+            mw[warp * 4 + c0] = m_run[0];
+            mw[warp * 4 + c1] = m_run[1];
+            lw[warp * 4 + c0] = l_run[0];
+            lw[warp * 4 + c1] = l_run[1];
+            dw[warp * 4 + c0] = dt_run[0];
+            dw[warp * 4 + c1] = dt_run[1];
+        }
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = mt * 16 + (lane >> 2) + ((r >> 1) << 3);
+                const int col = 2 * (lane & 3) + (r & 1);
+                float* dst = (col < 4) ? ap + (warp * 4 + col) * D : an + (warp * 4 + col - 4) * D;
+                dst[j] = acc[mt][r];
+            }
+    }
+    __syncthreads();
+    // merge the consumer warps and write the partial records
+    {
+        const float* mw = reinterpret_cast<const float*>(stages);
+        const float* lw = mw + NCW * 4;
+        const float* dw = lw + NCW * 4;
+        const float* ap = dw + NCW * 4;
+        const float* an = ap + NCW * 4 * D;
+        for (int e = tid; e < G * D; e += blockDim.x) {
+            const int g = e / D, j = e % D;
+            float M = -SPLA_INF;
+            for (int w = 0; w < NCW; ++w) M = fmaxf(M, mw[w * 4 + g]);
+            float l = 0.f, o = 0.f, nt = 0.f, dt = 0.f;
+            for (int w = 0; w < NCW; ++w) {
+                const float f = (M == -SPLA_INF) ? 0.f : ex2(mw[w * 4 + g] - M);
+                l += lw[w * 4 + g] * f;
+                o += ap[(w * 4 + g) * D + j] * f;
+                nt += an[(w * 4 + g) * D + j];
+                dt += dw[w * 4 + g];
+            }
+            float* rec = part + (rec_base + g) * REC;
+            rec[4 + j] = o;
+            rec[4 + D + j] = nsl[g * D + j] - nt;
+            if (j == 0) {
+                rec[0] = M;
+                rec[1] = l;
+                rec[2] = dsl[g] - dt;
+                rec[3] = 0.f;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ fp32 SIMT kernel
+// One CTA of 256 threads per (split, group). Tiles are staged through shared
+// memory as fp32; every product and sum is an fp32 FMA.
+template <typename T>
+__global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const T* __restrict__ q,
+                                                          float sl2,
+                                                          const uint32_t* __restrict__ bits,
+                                                          int nw, float* __restrict__ part,
+                                                          int nsplit, int max_per,
+                                                          int32_t* status) {
+    extern __shared__ __align__(16) unsigned char smem_simt[];
+    const int d = c.d, BS = c.bs, G = c.group;
+    float* Ks = reinterpret_cast<float*>(smem_simt);        // [BS][d]
+    float* Vs = Ks + BS * d;                                // [BS][d]
+    float* Ls = Vs + BS * d;                                // [4][BS] logits, then p
+    float* Ws = Ls + 4 * BS;                                // [4][BS] phi weights
+    float* qs = Ws + 4 * BS;                                // [4][d]
+    float* aw = qs + 4 * d;                                 // [4][d]
+    float* ml = aw + 4 * d;                                 // [d]
+    float* nsl = ml + d;                                    // [4][d]
+    float* dsl = nsl + 4 * d;                               // [4]
+    float* cg = dsl + 4;                                    // [4]
+    float* fsc = cg + 4;                                    // [4] per-head rescale of this tile
+    int32_t* blk = reinterpret_cast<int32_t*>(fsc + 4);
+    int32_t* phys = blk + max_per;
+    uint32_t* hm = reinterpret_cast<uint32_t*>(phys + max_per);
+    __shared__ int s_nblk;
+    __shared__ float s_m[4], s_l[4], s_dt[4];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv, split = blockIdx.x;
+    int32_t L = c.lens[b];
+    if (L < 0 || L > c.mbp * c.bs) L = max(0, min(L, c.mbp * c.bs));
+    const int nb = (L + BS - 1) / BS;
+    const int64_t rec_base = (((int64_t)b * c.hkv + h) * nsplit + split) * G;
+    const int REC = rec_floats(d);
+    if (nb == 0) {
+        for (int e = tid; e < G * REC; e += blockDim.x) {
+            const int g = e / REC, f = e % REC;
+            part[(rec_base + g) * REC + f] = (f == 0) ? -SPLA_INF : 0.f;
+        }
+        return;
+    }
+    if (warp == 0) {
+        const int n = build_union_share(c, bits, nw, b, h, nb, split, nsplit, max_per, blk, phys,
+                                        hm, status);
+        if (lane == 0) s_nblk = n;
+    }
+    query_setup(c, q, sizeof(T) == 2 ? SPLA_BF16 : SPLA_F32, b, h, qs, aw, ml, cg, tid, blockDim.x);
+    __syncthreads();
+    query_weights(c, b, h, qs, aw, cg, tid, blockDim.x);
+    __syncthreads();
+    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
+    for (int e = tid; e < G * d; e += blockDim.x) aw[e] = expf(qs[e] + mrow[e % d] - cg[e / d]);
+    if (tid < 4) { s_m[tid] = -SPLA_INF; s_l[tid] = 0.f; s_dt[tid] = 0.f; }
+    __syncthreads();
+    const int r0 = (int)((int64_t)split * d / nsplit), r1 = (int)((int64_t)(split + 1) * d / nsplit);
+    const float* Sg = c.S + ((int64_t)b * c.hkv + h) * d * d;
+    const float* zg = c.z + ((int64_t)b * c.hkv + h) * d;
+    for (int e = tid; e < G * d; e += blockDim.x) {
+        const int g = e / d, j = e % d;
+        float s = 0.f;
+        for (int i = r0; i < r1; ++i) s = fmaf(aw[g * d + i], Sg[(int64_t)i * d + j], s);
+        nsl[e] = s;
+    }
+    if (warp < G) {
+        float s = 0.f;
+        for (int i = r0 + lane; i < r1; i += 32) s = fmaf(aw[warp * d + i], zg[i], s);
+        s = warp_sum(s);
+        if (lane == 0) dsl[warp] = s;
+    }
+    const int nblk = s_nblk;
+    // accumulators: thread owns (g, j) pairs e = tid + 256*u
+    constexpr int PU = 2;                                   // G*d <= 512
+    float acc[PU] = {0.f, 0.f}, ntl[PU] = {0.f, 0.f};
+    for (int it = 0; it < nblk; ++it) {
+        const int jblk = blk[it];
+        const int nvalid = min(BS, L - jblk * BS);
+        const uint32_t hmask = hm[it];
+        __syncthreads();
+        const T* kp = (const T*)c.k_pool + ((int64_t)phys[it] * c.hkv + h) * BS * d;
+        const T* vp = (const T*)c.v_pool + ((int64_t)phys[it] * c.hkv + h) * BS * d;
+        for (int e = tid; e < BS * d; e += blockDim.x) {
+            const bool ok = (e / d) < nvalid;
+            Ks[e] = ok ? to_f(kp[e]) : 0.f;
+            Vs[e] = ok ? to_f(vp[e]) : 0.f;
+        }
+        __syncthreads();
+        // logits and phi weights per (g, t); dimension order rotated by t (no bank conflicts)
+        for (int e = tid; e < 4 * BS; e += blockDim.x) {
+            const int g = e / BS, t = e % BS;
+            float lg = -SPLA_INF, w = 0.f;
+            if (g < G && t < nvalid && ((hmask >> g) & 1u)) {
+                float sacc = 0.f, wacc = 0.f;
+                for (int u = 0; u < d; ++u) {
+                    const int i = (u + t) % d;
+                    const float kv = Ks[t * d + i];
+                    sacc = fmaf(qs[g * d + i], kv, sacc);
+                    wacc = fmaf(aw[g * d + i], ex2(fmaf(kv, SPLA_LOG2E, -ml[i])), wacc);
+                }
+                lg = sacc * sl2;
+                w = wacc;
+            }
+            Ls[e] = lg;
+            Ws[e] = w;
+        }
+        __syncthreads();
+        // online softmax, one warp per head
+        if (warp < G) {
+            float mx = -SPLA_INF;
+            for (int t = lane; t < BS; t += 32) mx = fmaxf(mx, Ls[warp * BS + t]);
+            mx = warp_max(mx);
+            const float mo = s_m[warp];
+            const float mn = fmaxf(mo, mx);
+            const float f = (mn == -SPLA_INF) ? 1.f : ex2(mo - mn);
+            float ls = 0.f, ds = 0.f;
+            for (int t = lane; t < BS; t += 32) {
+                const float lv = Ls[warp * BS + t];
+                const float p = (lv == -SPLA_INF) ? 0.f : ex2(lv - mn);
+                Ls[warp * BS + t] = p;
+                ls += p;
+                ds += Ws[warp * BS + t];
+            }
+            ls = warp_sum(ls);
+            ds = warp_sum(ds);
+            if (lane == 0) {
+                s_m[warp] = mn;
+                s_l[warp] = s_l[warp] * f + ls;
+                s_dt[warp] += ds;
+                fsc[warp] = f;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < PU; ++u) {
+            const int e = tid + 256 * u;
+            if (e < G * d) {
+                const int g = e / d, j = e % d;
+                float a = acc[u] * fsc[g], n = ntl[u];
+                for (int t = 0; t < nvalid; ++t) {
+                    const float vv = Vs[t * d + j];
+                    a = fmaf(Ls[g * BS + t], vv, a);
+                    n = fmaf(Ws[g * BS + t], vv, n);
+                }
+                acc[u] = a;
+                ntl[u] = n;
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < PU; ++u) {
+        const int e = tid + 256 * u;
+        if (e < G * d) {
+            const int g = e / d, j = e % d;
+            float* rec = part + (rec_base + g) * REC;
+            rec[4 + j] = acc[u];
+            rec[4 + d + j] = nsl[e] - ntl[u];
+            if (j == 0) {
+                rec[0] = s_m[g];
+                rec[1] = s_l[g];
+                rec[2] = dsl[g] - s_dt[g];
+                rec[3] = 0.f;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ combine
+template <typename T>
+__global__ void __launch_bounds__(128) combine_kernel(CacheView c, const float* __restrict__ part,
+                                                      int nsplit, const int32_t* __restrict__ nsel,
+                                                      const float* __restrict__ gamma, float eps,
+                                                      int no_rla, T* __restrict__ out,
+                                                      float* __restrict__ o_sp,
+                                                      float* __restrict__ o_rl) {
+    const int d = c.d, G = c.group;
+    const int b = blockIdx.x / c.hq, hq = blockIdx.x % c.hq;
+    const int h = hq / G, g = hq % G;
+    const int REC = rec_floats(d);
+    __shared__ float red[4];
+    int32_t L = c.lens[b];
+    L = max(0, min(L, c.mbp * c.bs));
+    const int nb = (L + c.bs - 1) / c.bs;
+    const bool all_sel = nsel[(int64_t)b * c.hq + hq] >= nb;
+    const float* recs = part + (((int64_t)b * c.hkv + h) * nsplit * G) * REC;
+    auto rec = [&](int s) { return recs + ((int64_t)s * G + g) * REC; };
+    float M = -SPLA_INF;
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, rec(s)[0]);
+    float Dr = 0.f;
+    float lsum = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+        const float* r = rec(s);
+        lsum += (M == -SPLA_INF) ? 0.f : r[1] * ex2(r[0] - M);
+        Dr += r[2];
+    }
+    const bool rla_off = no_rla || all_sel || !(Dr > 0.f) || L == 0;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        float o = 0.f, R = 0.f;
+        for (int s = 0; s < nsplit; ++s) {
+            const float* r = rec(s);
+            if (M != -SPLA_INF) o += r[4 + j] * ex2(r[0] - M);
+            R += r[4 + d + j];
+        }
+        o = (lsum > 0.f) ? o / lsum : 0.f;
+        const float rl = rla_off ? 0.f : R / Dr;
+        // RMS over d
+        float sq = rl * rl;
+        sq = warp_sum(sq);
+        if (d > 32) {
+            if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
+            __syncthreads();
+            sq = 0.f;
+            for (int w = 0; w < (min((int)blockDim.x, d) + 31) / 32; ++w) sq += red[w];
+            __syncthreads();
+        }
+        const float inv = rsqrtf(sq / d + eps);
+        const float gm = gamma ? gamma[(int64_t)hq * d + j] : 1.f;
+        const int64_t oi = ((int64_t)b * c.hq + hq) * d + j;
+        out[oi] = from_f<T>(o + gm * rl * inv);
+        if (o_sp) o_sp[oi] = o;
+        if (o_rl) o_rl[oi] = rl;
+    }
+}
+
+// ------------------------------------------------------------------ host launchers
+template <int D, int BS, int STAGES>
+static size_t mma_smem_bytes(int max_per) {
+    using Cfg = MmaCfg<D, BS, STAGES>;
+    return 1024 + (size_t)STAGES * Cfg::STAGE_BYTES + 2 * STAGES * sizeof(uint64_t) +
+           3 * (size_t)max_per * 4 + (size_t)(4 * D * 2 + D + 4 * D + 8) * 4 + 64;
+}
+
+template <int D, int BS, int STAGES>
+static cudaError_t launch_mma_t(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const void* q, float sl2, const uint32_t* bits, int nw,
+                                float* part, int nsplit, int max_per, int32_t* status,
+                                cudaStream_t s) {
+    using Cfg = MmaCfg<D, BS, STAGES>;
+    const size_t smem = mma_smem_bytes<D, BS, STAGES>(max_per);
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D, BS, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(nsplit, c.batch * c.hkv);
+    decode_mma_kernel<D, BS, STAGES><<<grid, Cfg::THREADS, smem, s>>>(
+        c, tk, tv, (const __nv_bfloat16*)q, sl2, bits, nw, part, nsplit, max_per, status);
+    return cudaGetLastError();
+}
+
+size_t mma_smem_for(int d, int bs, int max_per) {
+    if (d == 128 && bs == 64) return mma_smem_bytes<128, 64, 4>(max_per);
+    if (d == 128 && bs == 128) return mma_smem_bytes<128, 128, 3>(max_per);
+    if (d == 64 && bs == 64) return mma_smem_bytes<64, 64, 4>(max_per);
+    return mma_smem_bytes<64, 128, 4>(max_per);
+}
+
+cudaError_t launch_decode_mma(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const void* q, float sl2, const uint32_t* bits, int nw, float* part,
+                              int nsplit, int max_per, int32_t* status, cudaStream_t s) {
+    if (c.d == 128 && c.bs == 64)
+        return launch_mma_t<128, 64, 4>(c, tk, tv, q, sl2, bits, nw, part, nsplit, max_per, status, s);
+    if (c.d == 128 && c.bs == 128)
+        return launch_mma_t<128, 128, 3>(c, tk, tv, q, sl2, bits, nw, part, nsplit, max_per, status, s);
+    if (c.d == 64 && c.bs == 64)
+        return launch_mma_t<64, 64, 4>(c, tk, tv, q, sl2, bits, nw, part, nsplit, max_per, status, s);
+    return launch_mma_t<64, 128, 4>(c, tk, tv, q, sl2, bits, nw, part, nsplit, max_per, status, s);
+}
+
+size_t simt_smem_for(int d, int bs, int max_per) {
+    return (size_t)(2 * bs * d + 8 * bs + 4 * d * 3 + d + 16) * 4 + 3 * (size_t)max_per * 4 + 64;
+}
+
+cudaError_t launch_decode_simt(const CacheView& c, int dtype, const void* q, float sl2,
+                               const uint32_t* bits, int nw, float* part, int nsplit, int max_per,
+                               int32_t* status, cudaStream_t s) {
+    const size_t smem = simt_smem_for(c.d, c.bs, max_per);
+    dim3 grid(nsplit, c.batch * c.hkv);
+    cudaError_t e;
+    if (dtype == SPLA_BF16) {
+        e = cudaFuncSetAttribute(decode_simt_kernel<__nv_bfloat16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        decode_simt_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(
+            c, (const __nv_bfloat16*)q, sl2, bits, nw, part, nsplit, max_per, status);
+    } else {
+        e = cudaFuncSetAttribute(decode_simt_kernel<float>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        decode_simt_kernel<float><<<grid, 256, smem, s>>>(c, (const float*)q, sl2, bits, nw, part,
+                                                          nsplit, max_per, status);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CacheView& c, int dtype, const float* part, int nsplit,
+                           const int32_t* nsel, const float* gamma, float eps, int no_rla,
+                           void* out, float* o_sp, float* o_rl, cudaStream_t s) {
+    const int threads = c.d;                                 // 64 or 128
+    if (dtype == SPLA_BF16)
+        combine_kernel<__nv_bfloat16><<<c.batch * c.hq, threads, 0, s>>>(
+            c, part, nsplit, nsel, gamma, eps, no_rla, (__nv_bfloat16*)out, o_sp, o_rl);
+    else
+        combine_kernel<float><<<c.batch * c.hq, threads, 0, s>>>(c, part, nsplit, nsel, gamma, eps,
+                                                                 no_rla, (float*)out, o_sp, o_rl);
+    return cudaGetLastError();
+}
+
+}  // namespace spla

@@ -1,0 +1,194 @@
+/*
+ * spla.h -- C ABI of the SPLA decode library (libspla.so), sm_100a (B200).
+ *
+ * The method is "SPLA: Block Sparse Plus Linear Attention for Long Context
+ * Modeling" (gist.science technical summary, sections 2.1-2.3). One decode
+ * step, for every query head:
+ *   a1  score every KV block with the log of the second-order Taylor estimate
+ *       n_j exp(q'.mu_j)(1 + 1/2 q'^T diag(sigma_j^2) q'), q' = q * softmax_scale
+ *       (section 2.1);
+ *   a2  keep the top_k blocks (plus sink/local blocks when asked for);
+ *   a3  exact softmax attention over the kept blocks (section 2, opening);
+ *   a4  residual linear attention over the blocks not kept, by subtraction:
+ *       o_rla = (N - N~)/(D - D~), N, D from the global state S, z and
+ *       N~, D~ from the kept blocks, feature map phi = exp (section 2.2);
+ *   a5  out = o_sparse + gamma * RMSNorm(o_rla) (section 2.3).
+ * The state a4 reads is kept current by spla_append_kv (a0).
+ *
+ * Conventions
+ *   Memory.   Every pointer argument is DEVICE memory owned by the caller,
+ *             unless a comment says "host". The library allocates nothing and
+ *             never synchronises; all work is enqueued on `stream` (a
+ *             cudaStream_t passed as void*; NULL = legacy default stream).
+ *   Errors.   Argument errors are returned synchronously, before any CUDA
+ *             call, and nothing is enqueued. Faults the kernels detect
+ *             (a block-table entry out of range, a length past the table's
+ *             capacity, a bounded wait that ran out) are OR-ed into
+ *             *dev_status as SPLA_DEV_* bits; the caller reads it after its
+ *             own synchronisation. Kernels never trap.
+ *   Shapes.   Hq = num_q_heads, Hkv = num_kv_heads, G = Hq/Hkv (1, 2 or 4),
+ *             d = head_dim (64 or 128), B = block_size (64 or 128).
+ *   Dtypes.   q, K, V and out share params->dtype (SPLA_F32 or SPLA_BF16);
+ *             block statistics and the linear-attention state are fp32.
+ */
+#ifndef SPLA_H
+#define SPLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPLA_API __attribute__((visibility("default")))
+#else
+#define SPLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPLA_OK = 0,
+    SPLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size or inconsistent shape */
+    SPLA_ERR_UNSUPPORTED = 2,   /* shape outside what the kernels implement */
+    SPLA_ERR_WORKSPACE = 3,     /* workspace null or smaller than spla_decode_workspace_size */
+    SPLA_ERR_CAPACITY = 4,      /* a host-known size exceeds a fixed limit */
+    SPLA_ERR_CUDA = 5           /* a CUDA runtime call failed; see spla_last_cuda_error() */
+} spla_status;
+
+/* Bits the kernels OR into *dev_status. */
+#define SPLA_DEV_BAD_BLOCK_TABLE 0x1   /* a block-table entry outside [0, num_phys_blocks) */
+#define SPLA_DEV_CAPACITY        0x2   /* a length or an append past max_blocks_per_seq*B */
+#define SPLA_DEV_TIMEOUT         0x4   /* a bounded wait on a TMA barrier ran out */
+#define SPLA_DEV_BAD_COUNT       0x8   /* n_new[b] outside [0, max_new] */
+
+typedef enum { SPLA_F32 = 0, SPLA_BF16 = 1 } spla_dtype;
+
+/* params->flags */
+#define SPLA_FLAG_NO_RLA      0x1u  /* "SPA" ablation of section 4: o_rla = 0, out = o_sparse */
+#define SPLA_FLAG_FIRST_ORDER 0x2u  /* mean-only score (first-order ablation of section 4) */
+
+/* Largest max_blocks_per_seq the selection kernel handles. */
+#define SPLA_MAX_BLOCKS_PER_SEQ 32768
+
+typedef struct {
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t head_dim;        /* 64 or 128 */
+    int32_t block_size;      /* 64 or 128 */
+    int32_t top_k;           /* >= 1 */
+    int32_t n_sink;          /* first n_sink blocks always kept (0 unless a workload asks) */
+    int32_t n_local;         /* last n_local blocks always kept */
+    int32_t dtype;           /* spla_dtype */
+    float softmax_scale;     /* <= 0: 1/sqrt(head_dim) */
+    float rms_eps;           /* <= 0: 1e-6 */
+    uint32_t flags;          /* SPLA_FLAG_* */
+} spla_params;
+
+/*
+ * The paged KV cache and its per-block statistics and global state. All
+ * buffers are caller-allocated device memory; spla_cache_init prepares them.
+ *   k_pool, v_pool : [num_phys_blocks][Hkv][B][d], params->dtype. Slots past a
+ *                    sequence's length may hold anything.
+ *   blk_stats      : [num_phys_blocks][Hkv][2][d] fp32: key mean, then key
+ *                    population variance, of the block's stored tokens.
+ *   S              : [batch][Hkv][d][d] fp32, sum_t exp(k_t - m) v_t^T
+ *   z, m           : [batch][Hkv][d] fp32, sum_t exp(k_t - m) and the running
+ *                    per-dimension max of k (the state's scaling).
+ *   block_table    : [batch][max_blocks_per_seq] int32, logical -> physical block.
+ *   context_lens   : [batch] int32 tokens held; advanced by spla_append_kv.
+ */
+typedef struct {
+    void* k_pool;
+    void* v_pool;
+    float* blk_stats;
+    float* S;
+    float* z;
+    float* m;
+    const int32_t* block_table;
+    int32_t* context_lens;
+    int32_t batch;
+    int32_t max_blocks_per_seq;
+    int32_t num_phys_blocks;
+} spla_cache;
+
+/*
+ * Empty every sequence: context_lens = 0, S = 0, z = 0, m = -inf.
+ * Pools and statistics are left as they are (slots are rewritten on append).
+ */
+SPLA_API spla_status spla_cache_init(const spla_params* params, const spla_cache* cache, void* stream);
+
+/*
+ * a0 -- append tokens and keep the block statistics and the global state current
+ * (section 2.1: mean and diagonal variance per block; section 2.2: the global
+ * linear-attention state accumulates phi(k) v^T and phi(k) over every token).
+ *   k_new, v_new : [batch][max_new][Hkv][d], params->dtype; sequence b uses
+ *                  its first n_new[b] rows.
+ *   n_new        : [batch] int32 (device), each in [0, max_new].
+ *   max_new      : host int, >= 0; bounds the launch grid.
+ *   dev_status   : int32 (device), OR-ed with SPLA_DEV_* bits; may be NULL.
+ * For every sequence: tokens go to slots context_lens[b] .. + n_new[b] - 1
+ * through block_table; the statistics of every block touched are recomputed
+ * from all of its tokens; m rises to cover the new keys, S and z are rescaled
+ * by exp(m_old - m_new) and the new tokens added; context_lens[b] advances.
+ * A sequence whose append would pass max_blocks_per_seq*B, or whose n_new is
+ * out of range, is left unchanged and flagged.
+ */
+SPLA_API spla_status spla_append_kv(const spla_params* params, const spla_cache* cache,
+                           const void* k_new, const void* v_new, const int32_t* n_new,
+                           int32_t max_new, int32_t* dev_status, void* stream);
+
+/*
+ * Bytes of scratch spla_decode needs for this shape (host-only, no CUDA call).
+ * The value depends only on its arguments.
+ */
+SPLA_API spla_status spla_decode_workspace_size(const spla_params* params, int32_t batch,
+                                       int32_t max_blocks_per_seq, size_t* bytes);
+
+/*
+ * a1..a5 -- one decode step for every (sequence, query head).
+ *   q          : [batch][Hq][d], params->dtype.
+ *   rms_gamma  : [Hq][d] fp32 RMSNorm scale, or NULL for ones.
+ *   out        : [batch][Hq][d], params->dtype.
+ *   sel_idx    : [batch][Hq][top_k + n_sink + n_local] int32 or NULL: the
+ *                blocks kept, ascending, padded with -1.
+ *   o_sparse_dbg, o_rla_dbg : [batch][Hq][d] fp32 or NULL: the two branches
+ *                before the combine.
+ *   workspace  : device scratch of >= spla_decode_workspace_size bytes,
+ *                256-byte aligned; its contents need no initialisation.
+ *   dev_status : int32 (device) or NULL.
+ * Decode attends over tokens [0, context_lens[b]). An empty sequence gives
+ * out = 0. o_rla is 0 when every block is kept, or when the residual
+ * denominator D - D~ is not positive in fp32 (the residual mass is below the
+ * state's resolution). Selection ties go to the lower block index.
+ */
+SPLA_API spla_status spla_decode(const spla_params* params, const spla_cache* cache, const void* q,
+                        const float* rms_gamma, void* out, int32_t* sel_idx,
+                        float* o_sparse_dbg, float* o_rla_dbg,
+                        void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, void* stream);
+
+/*
+ * Measurement hook (no part of the method). With n == 5, every later
+ * spla_decode call made from this host thread records events[0..4]
+ * (cudaEvent_t handles) on its stream: before the scoring kernel, after it,
+ * after the selection kernel, after the split-KV decode kernel and after the
+ * combine kernel. n == 0 turns it off. The handles are copied; the events stay
+ * the caller's. Returns SPLA_ERR_INVALID_ARG for any other n or a NULL array.
+ */
+SPLA_API spla_status spla_profile_events(void* const* events, int32_t n);
+
+/* Human-readable name of a status (static storage). */
+SPLA_API const char* spla_status_string(spla_status s);
+
+/* The cudaError_t of the last CUDA call that failed in this thread (0 if none). */
+SPLA_API int32_t spla_last_cuda_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+SPLA_API int32_t spla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPLA_H */

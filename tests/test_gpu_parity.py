@@ -1,0 +1,233 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Small workloads keep each configuration's structure (heads, head_dim, block
+size, top-k, sink/local, value distribution, paging) at lengths the oracle
+handles in seconds, with ragged last blocks, and compare every head. Full-size
+workloads run the launch configuration the benchmark times and compare a
+sample of (sequence, KV head) groups.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import feed as ofeed
+from oracle import spla_oracle as so
+from workloads import feed_gpu, gen
+
+from . import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return None if t is None else t.float().cpu().numpy()
+
+
+def gpu_decode(cache, q_np, gamma_np, w):
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q = torch.from_numpy(q_np).to(dt).cuda()
+    gamma = torch.from_numpy(gamma_np).float().cuda()
+    out, sel, osp, orl = cache.new_outputs(debug=True)
+    cache.decode(q, gamma, out, sel, osp, orl)
+    torch.cuda.synchronize()
+    return dict(out=_np(out), sel=sel.cpu().numpy(), o_sparse=_np(osp), o_rla=_np(orl))
+
+
+def compare_all(res, oc, q, gamma, w, heads=None):
+    stats = []
+    p = oc.p
+    if heads is None:
+        heads = [(b, hq) for (b, h) in oc.state for hq in range(h * p.group, (h + 1) * p.group)]
+    for (b, hq) in heads:
+        g = {k: v[b, hq] for k, v in res.items()}
+        stats.append(parity.compare_head(g, oc, q, gamma, b, hq, w.dtype))
+    return stats
+
+
+def _summary(stats):
+    return dict(heads=len(stats), ties=sum(s["ties"] for s in stats),
+                ill=sum(not s["conditioned"] for s in stats),
+                max_sparse=max(s["e_sparse"] for s in stats),
+                max_out=max((s["e_out"] or 0) for s in stats))
+
+
+SMALL = {
+    "cfg1": dict(context_lens=(4096,)),
+    "cfg2": dict(context_lens=(4096 + 37, 3001)),
+    "cfg3": dict(context_lens=(8192 + 5, 6000)),
+    "cfg4": dict(context_lens=(65536 + 77,)),
+    "cfg5": dict(context_lens=(5000, 300, 12000, 64)),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_workload_matches_oracle(name):
+    w = gen.scaled(name, **SMALL[name])
+    cache = feed_gpu.build_cache(w)
+    oc = ofeed.build(w)
+    q = gen.query(w, 0)
+    gamma = gen.gamma(w, "random")
+    res = gpu_decode(cache, q, gamma, w)
+    st = compare_all(res, oc, q, gamma, w)
+    assert cache.status() == 0
+    s = _summary(st)
+    print(name, s)
+    assert s["ill"] <= s["heads"] // 4
+
+
+def test_interleaved_append_and_decode_match_oracle():
+    """Several steps of (append one token per sequence, decode), as the 128K workload runs."""
+    w = gen.scaled("cfg3", context_lens=(4096 - 2, 2047), plant_new_prob=0.5)
+    cache = feed_gpu.build_cache(w)
+    oc = ofeed.build(w)
+    gamma = gen.gamma(w)
+    for step in range(5):
+        k, v, qt = feed_gpu.step_inputs(w, step)
+        cache.append(k, v)
+        ofeed.append_step(oc, w, step)
+        q = gen.query(w, step)
+        res = gpu_decode(cache, q, gamma, w)
+        compare_all(res, oc, q, gamma, w)
+    assert cache.status() == 0
+    lens = cache.context_lens.cpu().numpy()
+    assert lens.tolist() == [4094 + 5, 2047 + 5]
+
+
+def test_append_state_matches_oracle():
+    """Block statistics and the scaled state after chunked prefill plus single-token appends."""
+    w = gen.scaled("cfg5", context_lens=(3000, 130, 9000))
+    cache = feed_gpu.build_cache(w)
+    oc = ofeed.build(w)
+    for step in range(3):
+        k, v, _ = feed_gpu.step_inputs(w, step)
+        cache.append(k, v)
+        ofeed.append_step(oc, w, step)
+    torch.cuda.synchronize()
+    table = gen.block_table(w)
+    stats = cache.blk_stats.cpu().numpy()
+    S, z, m = (t.cpu().numpy().astype(np.float64) for t in (cache.S, cache.z, cache.m))
+    for (b, h), g in oc.state.items():
+        np.testing.assert_array_equal(m[b, h], g.m)          # max of bf16 values: exact
+        np.testing.assert_allclose(z[b, h], g.z, rtol=2e-5)
+        np.testing.assert_allclose(S[b, h], g.S, rtol=2e-5, atol=2e-5 * np.abs(g.S).max())
+        n, mean, var = so.block_stats(g.K, w.block_size)
+        for j in range(len(n)):
+            st = stats[table[b, j], h]
+            np.testing.assert_allclose(st[0], mean[j], rtol=1e-6, atol=1e-7)
+            np.testing.assert_allclose(st[1], var[j], rtol=1e-6, atol=1e-7)
+
+
+# ----------------------------------------------------------------------------- edge cases
+def _tiny(**kw):
+    base = dict(context_lens=(700, 64, 1, 129))
+    base.update(kw)
+    return gen.scaled("cfg2", **base)
+
+
+def test_edge_lengths_tail_blocks_sink_local():
+    """Lengths 1, exactly one block, partial tails; sink and local blocks forced."""
+    w = _tiny()
+    cache = feed_gpu.build_cache(w)
+    oc = ofeed.build(w)
+    q, gamma = gen.query(w, 0), gen.gamma(w, "random")
+    res = gpu_decode(cache, q, gamma, w)
+    compare_all(res, oc, q, gamma, w)
+    assert cache.status() == 0
+
+
+def test_all_blocks_selected_gives_zero_rla():
+    """top_k >= blocks: o_rla is exactly zero and out equals o_sparse up to bf16 rounding."""
+    w = gen.scaled("cfg3", context_lens=(900, 64 * 5), top_k=64)
+    cache = feed_gpu.build_cache(w)
+    oc = ofeed.build(w)
+    q, gamma = gen.query(w, 0), gen.gamma(w)
+    res = gpu_decode(cache, q, gamma, w)
+    assert np.all(res["o_rla"] == 0)
+    compare_all(res, oc, q, gamma, w)
+
+
+def test_empty_sequence_in_batch_gives_zero():
+    w = gen.scaled("cfg3", context_lens=(1000, 0, 200))
+    cache = feed_gpu.build_cache(w)
+    q, gamma = gen.query(w, 0), gen.gamma(w)
+    res = gpu_decode(cache, q, gamma, w)
+    assert np.all(res["out"][1] == 0) and np.all(res["sel"][1] == -1)
+    oc = ofeed.build(w, groups=[(0, 0), (2, 3)])
+    compare_all(res, oc, q, gamma, w)
+
+
+@pytest.mark.parametrize("flag", ["no_rla", "first_order"])
+def test_ablation_flags_match_oracle(flag):
+    w = gen.scaled("cfg2", context_lens=(3000, 2000))
+    cache = feed_gpu.build_cache(w, cfg=feed_gpu.config_of(w, **{flag: True}))
+    oc = ofeed.build(w, **{flag: True})
+    q, gamma = gen.query(w, 0), gen.gamma(w)
+    res = gpu_decode(cache, q, gamma, w)
+    compare_all(res, oc, q, gamma, w)
+    if flag == "no_rla":
+        assert np.all(res["o_rla"] == 0)
+
+
+def test_fp32_path_head_dim_128_block_128():
+    """The fp32 kernel at the larger tile shape."""
+    w = gen.scaled("cfg4", context_lens=(5000, 2100), dtype="f32", top_k=8)
+    cache = feed_gpu.build_cache(w)
+    oc = ofeed.build(w)
+    q, gamma = gen.query(w, 0), gen.gamma(w, "random")
+    res = gpu_decode(cache, q, gamma, w)
+    compare_all(res, oc, q, gamma, w)
+
+
+def test_bad_block_table_entry_is_flagged_not_faulted():
+    """An out-of-range physical block id: kernels skip it and set the status bit."""
+    w = gen.scaled("cfg3", context_lens=(2000, 2000))
+    cache = feed_gpu.build_cache(w)
+    cache.block_table[1, 3] = w.num_phys_blocks + 5
+    q = torch.from_numpy(gen.query(w, 0)).to(torch.bfloat16).cuda()
+    cache.decode(q)
+    torch.cuda.synchronize()
+    assert cache.status() & 0x1
+
+
+def test_append_past_capacity_is_flagged():
+    w = gen.scaled("cfg3", context_lens=(300, 100), extra_tokens=0)
+    cache = feed_gpu.build_cache(w)
+    before = cache.context_lens.cpu().numpy().copy()
+    n = w.capacity_blocks * w.block_size - 300 + 1          # one token too many for seq 0
+    k = torch.zeros((2, n, w.num_kv_heads, w.head_dim), dtype=torch.bfloat16, device="cuda")
+    cache.append(k, k.clone(), torch.tensor([n, 1], dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert cache.status() & 0x2
+    after = cache.context_lens.cpu().numpy()
+    assert after[0] == before[0] and after[1] == before[1] + 1
+
+
+# ----------------------------------------------------------------------------- full size
+FULL_SAMPLE = {
+    "cfg1": None,                      # small enough: every head
+    "cfg2": [(0, 0), (5, 7)],
+    "cfg3": [(1, 2), (3, 5)],
+    "cfg4": [(0, 1), (0, 6)],
+    "cfg5": [(2, 0), (7, 4), (12, 3)],
+}
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", list(FULL_SAMPLE))
+def test_full_size_sampled_heads_match_oracle(name):
+    w = gen.get(name)
+    cache = feed_gpu.build_cache(w)
+    groups = FULL_SAMPLE[name]
+    oc = ofeed.build(w, groups=groups)
+    gamma = gen.gamma(w)
+    steps = 2 if name == "cfg3" else 1
+    for step in range(steps):
+        if name == "cfg3":
+            k, v, _ = feed_gpu.step_inputs(w, step)
+            cache.append(k, v)
+            ofeed.append_step(oc, w, step)
+        q = gen.query(w, step)
+        res = gpu_decode(cache, q, gamma, w)
+        st = compare_all(res, oc, q, gamma, w)
+        print(name, step, _summary(st))
+    assert cache.status() == 0
