@@ -10,7 +10,7 @@ Default workload: batch 4, 32 query / 8 KV heads, d 128, 131072-token
 contexts in 64-token blocks, top-k 32, 64 steps of append + decode (the
 128K-context decode workload). Inputs are synthetic and seeded
 (workloads/gen.py) and resident in HBM before timing; L2 is flushed (a
-512 MiB write) before every timed step and the flush is outside the events.
+512 MiB read) before every timed step and the flush is outside the events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg3]
     python bench.py --impl reference      # the CPU oracle on the host cores
@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="cfg3")
+    ap.add_argument("--context", type=int, default=0,
+                    help="profiling only: same workload at another context length")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -61,58 +63,66 @@ def peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples during the timed region (200 ms period)."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """NVML samples of SM clock and clock-event reasons every 2 ms during the timed region."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, index: int):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.index]) if vis else self.index
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         except Exception:
-            self.proc = None
+            self.nv = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self._stop.set()
+        if self.nv is not None:
             self.t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [x for x, _ in self.samples]
+        reasons = sorted(n for n, bit in self.REASONS.items()
+                         if any(r & bit for _, r in self.samples))
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm), "source": "NVML, 2 ms period"}
+
+
+class L2Flush:
+    """Evict L2 by reading 512 MiB (a read leaves no dirty lines for the next kernel)."""
+
+    def __init__(self, dev):
+        import torch
+        self.buf = torch.ones(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        self.acc = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        import torch
+        torch.sum(self.buf, out=self.acc)
 
 
 # ----------------------------------------------------------------------------- bytes
@@ -135,6 +145,14 @@ def step_bytes(w, sel: np.ndarray, lens: np.ndarray) -> dict:
     return {"kv": kv, "stats": stats, "state": state, "total": kv + stats + state}
 
 
+def workload_of(args):
+    from workloads import gen
+    if args.context > 0:
+        w = gen.get(args.workload)
+        return gen.scaled(args.workload, (args.context,) * w.batch, name=w.name)
+    return gen.get(args.workload)
+
+
 # ----------------------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -151,7 +169,7 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
-    w = gen.get(args.workload)
+    w = workload_of(args)
     K, W = args.steps, args.warmup
     cache = feed_gpu.build_cache(w, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -161,7 +179,7 @@ def run_ours(args):
     sels = torch.empty((2 * K, w.batch, w.num_q_heads, w.top_k + w.n_sink + w.n_local),
                        dtype=torch.int32, device=dev)
     lens_after = []
-    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    flush = L2Flush(dev)
 
     def step(s, sel=None):
         k, v, q = steps[s]
@@ -183,7 +201,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
         for i in range(K):
-            flush.zero_()
+            flush()
             ev0[i].record(stream)
             step(W + i, sels[i])
             ev1[i].record(stream)
@@ -200,7 +218,7 @@ def run_ours(args):
             e.record(stream)                  # materialise the handles
     torch.cuda.synchronize(dev)
     for i in range(K):
-        flush.zero_()
+        flush()
         _lib.spla_profile_events([e.cuda_event for e in pe[i]])
         step(W + K + i, sels[K + i])
     _lib.spla_profile_events([])
@@ -256,7 +274,7 @@ def run_ours(args):
                        "kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
                        "block": w.block_size, "top_k": w.top_k,
                        "step": "spla_append_kv (1 token/seq) + spla_decode",
-                       "l2": "flushed (512 MiB write) before every timed step, outside the events",
+                       "l2": "flushed (512 MiB read) before every timed step, outside the events",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": {"bound": "hbm", "kernel": kernel_names[dom],
                          "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
@@ -306,7 +324,7 @@ def e2e_pass(w, cache, steps, s0, K, gamma, flush, dev, stream):
     e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     torch.cuda.synchronize(dev)
     for i in range(K):
-        flush.zero_()
+        flush()
         e0[i].record(stream)
         hk, hv, hq = host[i]
         dk.copy_(hk, non_blocking=True)
@@ -365,7 +383,7 @@ def run_reference(args):
     if rank != 0:
         return
     from workloads import gen
-    w = gen.get(args.workload)
+    w = workload_of(args)
     oracle_sample(w, 0.0, steps=args.warmup)                  # warm-up (untimed)
     v, units, secs, desc, n = oracle_sample(w, 0.0, steps=args.steps)
     res = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT,

@@ -206,8 +206,6 @@ spla_status spla_append_kv(const spla_params* params, const spla_cache* cache, c
     if ((st = check_cache(cache)) != SPLA_OK) return st;
     if (max_new < 0 || !n_new) return SPLA_ERR_INVALID_ARG;
     if (max_new > 0 && (!k_new || !v_new)) return SPLA_ERR_INVALID_ARG;
-    if ((int64_t)max_new > (int64_t)cache->max_blocks_per_seq * params->block_size)
-        return SPLA_ERR_CAPACITY;
     const CacheView v = view_of(params, cache);
     cudaError_t e = launch_append(v, params->dtype, k_new, v_new, n_new, max_new, dev_status,
                                   (cudaStream_t)stream);

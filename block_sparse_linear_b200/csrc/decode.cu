@@ -153,7 +153,9 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     int32_t* blk = reinterpret_cast<int32_t*>(empty + STAGES);
     int32_t* phys = blk + max_per;
     uint32_t* hm = reinterpret_cast<uint32_t*>(phys + max_per);
-    float* qs = reinterpret_cast<float*>(hm + max_per);     // [4][D]
+    // 16-byte aligned: ml is read as float2 (max_per may be odd)
+    float* qs = reinterpret_cast<float*>(
+        (reinterpret_cast<uintptr_t>(hm + max_per) + 15) & ~uintptr_t(15));   // [4][D]
     float* aw = qs + G4 * D;                                // [4][D]
     float* ml = aw + G4 * D;                                // [D]
     float* nsl = ml + D;                                    // [4][D]
@@ -706,7 +708,7 @@ template <int D, int BS, int STAGES>
 static size_t mma_smem_bytes(int max_per) {
     using Cfg = MmaCfg<D, BS, STAGES>;
     return 1024 + (size_t)STAGES * Cfg::STAGE_BYTES + 2 * STAGES * sizeof(uint64_t) +
-           3 * (size_t)max_per * 4 + (size_t)(4 * D * 2 + D + 4 * D + 8) * 4 + 64;
+           3 * (size_t)max_per * 4 + 16 + (size_t)(4 * D * 2 + D + 4 * D + 8) * 4 + 64;
 }
 
 template <int D, int BS, int STAGES>

@@ -6,7 +6,10 @@ Acceptance, per (sequence, query head):
   (relative 1e-6 on the linear score is 1e-6 absolute on its log);
 * outputs: the oracle is re-run on the GPU's own selection; o_sparse, o_rla
   and out must match within 1e-4 * max(1, max|ref|) for fp32 workloads and
-  2e-2 absolute for bf16 workloads.
+  2e-2 absolute for bf16 workloads. o_sparse and o_rla come back in fp32; out
+  comes back in bf16 for bf16 workloads, so its bound also allows the output
+  format's own rounding, half a bf16 ulp of the reference value (|out| >= 8
+  has an ulp of 0.0625, beyond 2e-2 for any bf16 number).
 o_rla and out are compared only where the RLA subtraction is well
 conditioned: kappa = max(D/(D - D~), |N|_inf/|N - N~|_inf), computed by the
 oracle in fp64, bounds how much the fp32 state's rounding is amplified. Heads
@@ -19,6 +22,12 @@ from oracle import spla_oracle as so
 SEL_TIE = 1e-6
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 KAPPA_MAX = {"f32": 10.0, "bf16": 2e3}
+
+
+def bf16_ulp(x):
+    """Spacing of bf16 numbers at |x| (8 significand bits)."""
+    ax = np.maximum(np.abs(np.asarray(x, np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(ax)) - 7)
 
 
 def kappa(q, g: so.GroupState, p: so.OracleParams, sel) -> float:
@@ -70,7 +79,11 @@ def compare_head(gpu: dict, oc: so.OracleCache, q, gamma, b, hq, dtype: str) -> 
     def err(name):
         r = fref[name]
         scale = max(1.0, float(np.abs(r).max())) if dtype == "f32" else 1.0
-        return float(np.abs(np.asarray(gpu[name], np.float64) - r).max()) / scale
+        d = np.abs(np.asarray(gpu[name], np.float64) - r)
+        if name == "out" and dtype == "bf16":
+            # the output format's own rounding (half a bf16 ulp of the value) comes on top
+            d = np.maximum(d - 0.5 * bf16_ulp(r), 0.0)
+        return float(d.max()) / scale
 
     e_sp = err("o_sparse")
     assert e_sp <= tol, f"o_sparse ({b},{hq}) err {e_sp:.3g} > {tol}"

@@ -114,8 +114,6 @@ def test_bad_cache_and_buffers_rejected(lib):
         _lib.SPLA_ERR_INVALID_ARG
     assert lib.spla_append_kv(B(p), B(c), FAKE, FAKE, None, 4, None, None) == \
         _lib.SPLA_ERR_INVALID_ARG
-    assert lib.spla_append_kv(B(p), B(c), FAKE, FAKE, FAKE, 2064 * 64 + 1, None, None) == \
-        _lib.SPLA_ERR_CAPACITY
 
 
 def test_python_binding_raises_on_error_codes():

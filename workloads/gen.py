@@ -150,8 +150,8 @@ def get(name: str, **overrides) -> Workload:
 def scaled(name: str, context_lens, **overrides) -> Workload:
     """The named workload's structure (heads, d, block, top-k, distributions) at other lengths."""
     lens = tuple(int(x) for x in context_lens)
-    return replace(CONFIGS[name], context_lens=lens, batch=len(lens), name=f"{name}-small",
-                   **overrides)
+    overrides.setdefault("name", f"{name}-small")
+    return replace(CONFIGS[name], context_lens=lens, batch=len(lens), **overrides)
 
 
 # --------------------------------------------------------------------------- rng helpers
