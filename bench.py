@@ -122,7 +122,7 @@ class L2Flush:
 
     def __call__(self):
         import torch
-        torch.sum(self.buf, out=self.acc)
+        torch.sum(self.buf, 0, out=self.acc)
 
 
 # ----------------------------------------------------------------------------- bytes

@@ -16,21 +16,18 @@ cudaError_t launch_score(const CacheView& c, int dtype, const void* q, double sc
                          cudaStream_t s);
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
                           const float* scores, uint32_t* bits, int nw, int32_t* nsel,
-                          int32_t* sel_idx, int kcap, cudaStream_t s);
+                          int32_t* sel_idx, int kcap, int32_t* counters, cudaStream_t s);
 cudaError_t launch_decode_mma(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
-                              const void* q, float sl2, const uint32_t* bits, int nw, float* part,
-                              int nsplit, int max_per, int32_t* status, cudaStream_t s);
-cudaError_t launch_decode_simt(const CacheView& c, int dtype, const void* q, float sl2,
-                               const uint32_t* bits, int nw, float* part, int nsplit, int max_per,
-                               int32_t* status, cudaStream_t s);
-cudaError_t launch_combine(const CacheView& c, int dtype, const float* part, int nsplit,
-                           const int32_t* nsel, const float* gamma, float eps, int no_rla,
-                           void* out, float* o_sp, float* o_rl, cudaStream_t s);
+                              const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_simt(const CacheView& c, int dtype, const DecodeArgs& a, cudaStream_t s);
 size_t mma_smem_for(int d, int bs, int max_per);
 size_t simt_smem_for(int d, int bs, int max_per);
 
-// The split heuristic is tuned for the 148-SM B200; results do not depend on it.
+// The split heuristic is tuned for the 148-SM B200 (two decode CTAs per SM);
+// results do not depend on it.
 constexpr int kTargetCtas = 148;
+constexpr int kDecodeSlots = 2 * kTargetCtas;
+constexpr int kMaxSplit = 512;
 constexpr int kMaxSmem = 227 * 1024;
 
 static thread_local int32_t g_last_cuda_error = 0;
@@ -102,13 +99,15 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     L.nw = (mbp + 31) / 32;
     L.rec = rec_floats(p->head_dim);
     const int umax = (int)std::min<int64_t>(mbp, (int64_t)G * L.kcap);
-    int ns = (kTargetCtas + groups - 1) / groups;       // enough CTAs to cover the SMs once
-    ns = std::max(1, std::min(ns, std::max(1, umax / 2)));
+    // one wave: as many splits per group as fit the resident CTA slots, at least 2 blocks each
+    int ns = kDecodeSlots / groups;
+    ns = std::max(1, std::min(ns, std::min(kMaxSplit, std::max(1, umax / 2))));
     L.nsplit = ns;
     L.max_per = (umax + ns - 1) / ns + 1;
-    // scoring chunk: enough CTAs to fill the machine twice over
-    int chunk = 256;
-    while (chunk > 64 && (int64_t)groups * ((mbp + chunk - 1) / chunk) < 2 * kTargetCtas) chunk >>= 1;
+    // scoring chunk: 128 blocks per CTA (one pass of its 4 warps); smaller if that
+    // leaves fewer than four CTAs per SM
+    int chunk = 128;
+    while (chunk > 32 && (int64_t)groups * ((mbp + chunk - 1) / chunk) < 4 * kTargetCtas) chunk >>= 1;
     L.score_chunk = chunk;
     size_t off = 0;
     L.off_scores = off;
@@ -119,6 +118,8 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     off = align256(off + (size_t)batch * p->num_q_heads * sizeof(int32_t));
     L.off_part = off;
     off = align256(off + (size_t)groups * ns * G * L.rec * sizeof(float));
+    L.off_cnt = off;
+    off = align256(off + (size_t)groups * sizeof(int32_t));
     L.total = off;
     return L;
 }
@@ -138,14 +139,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D view of a pool as [num_phys*Hkv*B rows][d cols] bf16; box = B rows x 64 cols, 128B swizzle.
+// 2-D view of a pool as [num_phys*Hkv*B rows][d cols] bf16; box = 64 rows x 64 cols (one
+// 64-token pipeline unit of the decode kernel, 8 KiB), 128B swizzle.
 static bool make_pool_map(CUtensorMap* m, const void* pool, const CacheView& c) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t rows = (cuuint64_t)c.num_phys * c.hkv * c.bs;
     cuuint64_t dims[2] = {(cuuint64_t)c.d, rows};
     cuuint64_t strides[1] = {(cuuint64_t)c.d * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)c.bs};
+    cuuint32_t box[2] = {64u, 64u};
     cuuint32_t estr[2] = {1u, 1u};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -257,25 +259,38 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
                                  dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(1, s);
+    int32_t* counters = reinterpret_cast<int32_t*>(ws + L.off_cnt);
     e = launch_select(v, params->top_k, params->n_sink, params->n_local, scores, bits, L.nw, nsel,
-                      sel_idx, L.kcap, s);
+                      sel_idx, L.kcap, counters, s);
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(2, s);
+    DecodeArgs da;
+    da.q = q;
+    da.gamma = rms_gamma;
+    da.out = out;
+    da.o_sp = o_sparse_dbg;
+    da.o_rl = o_rla_dbg;
+    da.bits = bits;
+    da.nsel = nsel;
+    da.part = part;
+    da.counters = counters;
+    da.status = dev_status;
+    da.nw = L.nw;
+    da.nsplit = L.nsplit;
+    da.max_per = L.max_per;
+    da.no_rla = no_rla;
+    da.sl2 = sl2;
+    da.eps = eps;
     if (use_mma) {
         CUtensorMap tk, tv;
         if (!make_pool_map(&tk, v.k_pool, v) || !make_pool_map(&tv, v.v_pool, v))
             return cuda_fail(cudaErrorInvalidValue);
-        e = launch_decode_mma(v, tk, tv, q, sl2, bits, L.nw, part, L.nsplit, L.max_per, dev_status,
-                              s);
+        e = launch_decode_mma(v, tk, tv, da, s);
     } else {
-        e = launch_decode_simt(v, params->dtype, q, sl2, bits, L.nw, part, L.nsplit, L.max_per,
-                               dev_status, s);
+        e = launch_decode_simt(v, params->dtype, da, s);
     }
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(3, s);
-    e = launch_combine(v, params->dtype, part, L.nsplit, nsel, rms_gamma, eps, no_rla, out,
-                       o_sparse_dbg, o_rla_dbg, s);
-    if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(4, s);
     return SPLA_OK;
 }

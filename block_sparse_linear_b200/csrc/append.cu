@@ -6,7 +6,8 @@
 //
 // Three launches, stream-ordered:
 //   append_kv_stats  grid (touched blocks, batch*Hkv): write tokens, then the
-//                    block's mean and population variance in fp64 (two-pass);
+//                    block's mean and population variance in fp64 (two-pass,
+//                    keys staged in shared memory);
 //   append_state     grid (d/8 row groups, batch*Hkv): m <- max(m, k_new),
 //                    rescale S and z rows by exp(m_old - m_new), add
 //                    exp(k - m_new) v^T and exp(k - m_new);
@@ -64,20 +65,36 @@ __global__ void __launch_bounds__(256) append_kv_stats_kernel(CacheView c, const
         vp[(int64_t)(t - blk_lo) * d + i] = v_new[src];
     }
     __syncthreads();
-    // statistics over all tokens now in the block: two passes in fp64
+    // statistics over all tokens now in the block: stage the keys in shared
+    // memory with coalesced loads, then two passes per dimension in fp64
+    extern __shared__ float ktile[];                 // [nj][d]
     const int nj = t_end - (int)blk_lo;
+    for (int e = threadIdx.x; e < nj * d; e += blockDim.x) ktile[e] = to_f(kp[e]);
+    __syncthreads();
     float* st = c.stats + ((int64_t)phys * c.hkv + h) * 2 * d;
-    for (int i = threadIdx.x; i < d; i += blockDim.x) {
-        double s = 0.0;
-        for (int t = 0; t < nj; ++t) s += (double)to_f(kp[(int64_t)t * d + i]);
-        const double mean = s / nj;
-        double q = 0.0;
-        for (int t = 0; t < nj; ++t) {
-            const double x = (double)to_f(kp[(int64_t)t * d + i]) - mean;
-            q += x * x;
-        }
+    const int parts = blockDim.x / d;                // threads per dimension (2 at d=128, 4 at 64)
+    const int i = threadIdx.x % d, part = threadIdx.x / d;
+    __shared__ double red[256];
+    double s = 0.0;
+    for (int t = part; t < nj; t += parts) s += (double)ktile[t * d + i];
+    red[threadIdx.x] = s;
+    __syncthreads();
+    double tot = 0.0;
+    for (int p = 0; p < parts; ++p) tot += red[p * d + i];
+    const double mean = tot / nj;
+    __syncthreads();
+    double q = 0.0;
+    for (int t = part; t < nj; t += parts) {
+        const double x = (double)ktile[t * d + i] - mean;
+        q += x * x;
+    }
+    red[threadIdx.x] = q;
+    __syncthreads();
+    if (part == 0) {
+        double qt = 0.0;
+        for (int p = 0; p < parts; ++p) qt += red[p * d + i];
         st[i] = (float)mean;
-        st[d + i] = (float)(q / nj);
+        st[d + i] = (float)(qt / nj);
     }
 }
 
@@ -177,13 +194,22 @@ cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, cons
     if (max_new > 0) {
         dim3 g1((max_new + c.bs - 1) / c.bs + 1, c.batch * c.hkv);
         dim3 g2((c.d + 7) / 8, c.batch * c.hkv);
+        const size_t smem = (size_t)c.bs * c.d * sizeof(float);
+        if (smem > 48 * 1024) {
+            cudaError_t e = dtype == SPLA_BF16
+                ? cudaFuncSetAttribute(append_kv_stats_kernel<__nv_bfloat16>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                : cudaFuncSetAttribute(append_kv_stats_kernel<float>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
         if (dtype == SPLA_BF16) {
-            append_kv_stats_kernel<__nv_bfloat16><<<g1, 256, 0, s>>>(
+            append_kv_stats_kernel<__nv_bfloat16><<<g1, 256, smem, s>>>(
                 c, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_new, max_new, status);
             append_state_kernel<__nv_bfloat16><<<g2, 256, 0, s>>>(
                 c, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_new, max_new);
         } else {
-            append_kv_stats_kernel<float><<<g1, 256, 0, s>>>(c, (const float*)k_new,
+            append_kv_stats_kernel<float><<<g1, 256, smem, s>>>(c, (const float*)k_new,
                                                             (const float*)v_new, n_new, max_new,
                                                             status);
             append_state_kernel<float><<<g2, 256, 0, s>>>(c, (const float*)k_new,

@@ -36,7 +36,23 @@ struct DecodeLayout {
     int32_t rec;             // floats per partial record
     int32_t score_chunk;     // blocks per scoring CTA
     int32_t max_per;         // union blocks one decode CTA may receive
-    size_t off_scores, off_bits, off_nsel, off_part, total;
+    size_t off_scores, off_bits, off_nsel, off_part, off_cnt, total;
+};
+
+// Per-call arguments of the decode kernels beyond the cache.
+struct DecodeArgs {
+    const void* q;
+    const float* gamma;         // [Hq][d] or null
+    void* out;                  // [batch][Hq][d], dtype
+    float* o_sp;                // [batch][Hq][d] or null
+    float* o_rl;                // [batch][Hq][d] or null
+    const uint32_t* bits;       // [batch][Hq][nw] selection bitsets
+    const int32_t* nsel;        // [batch][Hq]
+    float* part;                // [batch*Hkv][nsplit][G][rec]
+    int32_t* counters;          // [batch*Hkv], zeroed by the selection kernel
+    int32_t* status;
+    int nw, nsplit, max_per, no_rla;
+    float sl2, eps;
 };
 
 // Partial record of one decode CTA for one query head:

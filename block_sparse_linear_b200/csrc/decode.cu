@@ -1,5 +1,5 @@
 // a3 + a4 + a5 -- split-KV decode over the kept blocks with the residual linear
-// attention computed in the same pass, then the split combine (SPLA technical
+// attention computed in the same pass, and the split combine (SPLA technical
 // summary, gist.science: section 2 opening -- exact attention over the kept
 // blocks; section 2.2 -- RLA by subtraction, the kept blocks' linear-attention
 // term computed while they are on chip so unkept blocks are never read;
@@ -10,8 +10,8 @@
 //
 // Grid (nsplit, batch*Hkv). Every CTA of a (sequence, KV head) group:
 //   * forms the union of the G heads' selections from their bitsets and takes
-//     an equal share of it (the union is read once for all G heads; a head
-//     that did not select a block is masked out of that block);
+//     an equal share of it (a union block is read once for all G heads; a head
+//     that did not select it is masked out of it);
 //   * reads rows [s*d/nsplit, (s+1)*d/nsplit) of the state S, z and computes
 //     that slice of the global linear-attention readout N, D;
 //   * streams its blocks' K and V tiles and accumulates, per head, the online
@@ -19,17 +19,20 @@
 //     numerator and denominator (N~ = sum w v, D~ = sum w) with
 //     w_t = sum_i exp(q_i + m_i - c) exp(k_t,i - m_i);
 //   * writes one partial record per head: m, l, acc, R = N_slice - N~, Dr = D_slice - D~.
-// combine_kernel merges the records of a head: the log-sum-exp merge of the
-// softmax partials, o_rla = sum R / sum Dr, RMSNorm, out = o_sparse + gamma*RMSNorm(o_rla).
+// The last CTA of a group to finish (an atomic counter) merges the group's
+// records: log-sum-exp merge of the softmax partials, o_rla = sum R / sum Dr,
+// RMSNorm, out = o_sparse + gamma * RMSNorm(o_rla).
 //
-// decode_mma_kernel (bf16 K/V): 4 consumer warps + 1 TMA producer warp. Each
-// (block, KV head) K or V tile is fetched by 2-D tiled TMA (128-byte swizzle,
-// no multicast) into a STAGES-deep mbarrier ring. Per 16-token slab a warp
-// runs the G-head contractions on tensor cores (mma.sync m16n8k16 bf16):
+// decode_mma_kernel (bf16 K/V): 4 consumer warps + 1 TMA producer warp, two
+// CTAs per SM. The pipeline unit is a 64-token tile of one (block, KV head):
+// its K and V come by 2-D tiled TMA (128-byte swizzle, no multicast) into a
+// 3-deep mbarrier ring (a 128-token block is two units). Each consumer warp
+// owns one 16-token slab of a unit and runs the G-head contractions on tensor
+// cores (mma.sync m16n8k16 bf16, fp32 accumulate):
 //   logits  = K(16 x d) . Q^T(d x 8)            (q exact in bf16)
 //   w       = phi(K)(16 x d) . [a_hi a_lo]^T    (phi(K) split hi/lo in bf16)
 //   O^T    += V^T(d x 16) . [P W]_{hi,lo}       (P, W split hi/lo in bf16)
-// so every computed operand carries ~16 mantissa bits and sums are fp32.
+// so every computed operand carries ~16 mantissa bits.
 // decode_simt_kernel (fp32 or bf16 K/V): plain fp32 FMA, for the fp32 path.
 #include "common.cuh"
 
@@ -95,23 +98,24 @@ __device__ int build_union_share(const CacheView& c, const uint32_t* bits, int n
     return min(u1 - u0, max_per);
 }
 
-// Query-side constants (run by nthr threads with barrier id `bar`):
-//   qs[g][i] = q (fp32), a[g][i] = exp(q_i + m_i - c_g), ml[i] = m_i*log2e.
-__device__ void query_setup(const CacheView& c, const void* q, int dtype, int b, int h,
-                            float* qs, float* a, float* ml, float* cg, int tid, int nthr) {
+// Query-side constants, computed by nthr threads (tid in [0, nthr)); the caller
+// synchronises between the three steps:
+//   1) qs[g][i] = q (fp32), ml[i] = m_i * log2e
+//   2) cg[g] = max_i (q_i + m_i)                  (warps 0..G-1)
+//   3) aw[g][i] = exp(q_i + m_i - c_g)
+__device__ void query_load(const CacheView& c, const void* q, int is_bf16, int b, int h,
+                           float* qs, float* ml, int tid, int nthr) {
     const int G = c.group, d = c.d;
     const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
     for (int e = tid; e < G * d; e += nthr) {
         const int g = e / d, i = e % d;
         const int64_t qi = ((int64_t)b * c.hq + h * G + g) * d + i;
-        qs[e] = dtype == SPLA_BF16 ? __bfloat162float(((const __nv_bfloat16*)q)[qi])
-                                   : ((const float*)q)[qi];
+        qs[e] = is_bf16 ? __bfloat162float(((const __nv_bfloat16*)q)[qi]) : ((const float*)q)[qi];
     }
     for (int i = tid; i < d; i += nthr) ml[i] = mrow[i] * SPLA_LOG2E;
 }
 
-__device__ void query_weights(const CacheView& c, int b, int h, const float* qs, float* a,
-                              float* cg, int tid, int nthr) {
+__device__ void query_max(const CacheView& c, int b, int h, const float* qs, float* cg, int tid) {
     const int G = c.group, d = c.d;
     const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
     const int warp = tid >> 5, lane = tid & 31;
@@ -123,52 +127,186 @@ __device__ void query_weights(const CacheView& c, int b, int h, const float* qs,
     }
 }
 
+__device__ void query_phi(const CacheView& c, int b, int h, const float* qs, const float* cg,
+                          float* aw, int tid, int nthr) {
+    const int G = c.group, d = c.d;
+    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
+    for (int e = tid; e < G * d; e += nthr) aw[e] = expf(qs[e] + mrow[e % d] - cg[e / d]);
+}
+
+// Slice [r0, r1) of the global readout: nsl[g][j] = sum_i aw[g][i] S[i][j], dsl[g] = sum_i aw[g][i] z[i].
+__device__ void state_slice(const CacheView& c, int b, int h, int r0, int r1, const float* aw,
+                            float* nsl, float* dsl, int tid, int nthr) {
+    const int G = c.group, d = c.d;
+    const float* Sg = c.S + ((int64_t)b * c.hkv + h) * d * d;
+    const float* zg = c.z + ((int64_t)b * c.hkv + h) * d;
+    for (int j = tid; j < d; j += nthr) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int i = r0; i < r1; ++i) {
+            const float sv = Sg[(int64_t)i * d + j];
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                if (g < G) acc[g] = fmaf(aw[g * d + i], sv, acc[g]);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+            if (g < G) nsl[g * d + j] = acc[g];
+    }
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < G) {
+        float s = 0.f;
+        for (int i = r0 + lane; i < r1; i += 32) s = fmaf(aw[warp * d + i], zg[i], s);
+        s = warp_sum(s);
+        if (lane == 0) dsl[warp] = s;
+    }
+}
+
+// ------------------------------------------------------------------ group combine
+// Run by the last CTA of a (sequence, KV head) group. scr: >= 4*nsplit + 8*d + 32 floats.
+template <typename T>
+__device__ void combine_group(const CacheView& c, const DecodeArgs& a, int b, int h, float* scr,
+                              int tid, int nthr) {
+    const int G = c.group, d = c.d, REC = rec_floats(d), ns = a.nsplit;
+    const float* recs = a.part + ((int64_t)b * c.hkv + h) * ns * G * REC;   // [ns][G][REC]
+    float* sM = scr;            // [4]
+    float* sL = sM + 4;         // [4]
+    float* sD = sL + 4;         // [4]
+    float* sQ = sD + 4;         // [4] 1/rms of o_rla
+    float* fac = sQ + 4 + 16;   // [4][ns]
+    float* orl = fac + 4 * ns;  // [4][d]
+    float* osp = orl + 4 * d;   // [4][d]
+    const int warp = tid >> 5, lane = tid & 31;
+    int32_t L = c.lens[b];
+    L = max(0, min(L, c.mbp * c.bs));
+    const int nb = (L + c.bs - 1) / c.bs;
+    if (warp < G) {
+        const int g = warp;
+        float M = -SPLA_INF;
+        for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldcg(recs + ((int64_t)s * G + g) * REC));
+        M = warp_max(M);
+        float l = 0.f, dr = 0.f;
+        for (int s = lane; s < ns; s += 32) {
+            const float* r = recs + ((int64_t)s * G + g) * REC;
+            const float f = (M == -SPLA_INF) ? 0.f : ex2(__ldcg(r) - M);
+            fac[g * ns + s] = f;
+            l += __ldcg(r + 1) * f;
+            dr += __ldcg(r + 2);
+        }
+        l = warp_sum(l);
+        dr = warp_sum(dr);
+        if (lane == 0) {
+            sM[g] = M;
+            sL[g] = l;
+            sD[g] = dr;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < G * d; e += nthr) {
+        const int g = e / d, j = e % d;
+        float o0 = 0.f, o1 = 0.f, R0 = 0.f, R1 = 0.f;
+        int s = 0;
+        for (; s + 1 < ns; s += 2) {
+            const float* r = recs + ((int64_t)s * G + g) * REC;
+            const float* r2 = r + (int64_t)G * REC;
+            o0 = fmaf(__ldcg(r + 4 + j), fac[g * ns + s], o0);
+            o1 = fmaf(__ldcg(r2 + 4 + j), fac[g * ns + s + 1], o1);
+            R0 += __ldcg(r + 4 + d + j);
+            R1 += __ldcg(r2 + 4 + d + j);
+        }
+        if (s < ns) {
+            const float* r = recs + ((int64_t)s * G + g) * REC;
+            o0 = fmaf(__ldcg(r + 4 + j), fac[g * ns + s], o0);
+            R0 += __ldcg(r + 4 + d + j);
+        }
+        const float lsum = sL[g], Dr = sD[g];
+        const int hq = h * G + g;
+        const bool all_sel = a.nsel[(int64_t)b * c.hq + hq] >= nb;
+        const bool off = a.no_rla || all_sel || !(Dr > 0.f) || L == 0;
+        osp[e] = (lsum > 0.f) ? (o0 + o1) / lsum : 0.f;
+        orl[e] = off ? 0.f : (R0 + R1) / Dr;
+    }
+    __syncthreads();
+    if (warp < G) {
+        float sq = 0.f;
+        for (int j = lane; j < d; j += 32) sq = fmaf(orl[warp * d + j], orl[warp * d + j], sq);
+        sq = warp_sum(sq);
+        if (lane == 0) sQ[warp] = rsqrtf(sq / d + a.eps);
+    }
+    __syncthreads();
+    for (int e = tid; e < G * d; e += nthr) {
+        const int g = e / d, j = e % d;
+        const int hq = h * G + g;
+        const int64_t oi = ((int64_t)b * c.hq + hq) * d + j;
+        const float gm = a.gamma ? a.gamma[(int64_t)hq * d + j] : 1.f;
+        static_cast<T*>(a.out)[oi] = from_f<T>(osp[e] + gm * orl[e] * sQ[g]);
+        if (a.o_sp) a.o_sp[oi] = osp[e];
+        if (a.o_rl) a.o_rl[oi] = orl[e];
+    }
+}
+
+// Count this CTA in; the last one of the group combines (fence, then counter).
+template <typename T>
+__device__ void finish_group(const CacheView& c, const DecodeArgs& a, int b, int h, float* scr,
+                             int tid, int nthr, int* s_flag) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const int old = atomicAdd(&a.counters[(int64_t)b * c.hkv + h], 1);
+        *s_flag = (old == a.nsplit - 1);
+    }
+    __syncthreads();
+    if (*s_flag) {
+        __threadfence();
+        combine_group<T>(c, a, b, h, scr, tid, nthr);
+        if (tid == 0) a.counters[(int64_t)b * c.hkv + h] = 0;
+    }
+}
+
 // ------------------------------------------------------------------ bf16 tensor-core kernel
-template <int D, int BS, int STAGES>
+template <int D, int UPB, int STAGES>
 struct MmaCfg {
-    static constexpr int NCW = 4;                           // consumer warps
+    static constexpr int NCW = 4;                           // consumer warps (one slab each)
     static constexpr int THREADS = (NCW + 1) * 32;
+    static constexpr int BS = 64 * UPB;                     // tokens per block
     static constexpr int BOXES = D / 64;                    // 64-column boxes per tile
-    static constexpr int BOX_BYTES = BS * 128;
-    static constexpr int TILE_BYTES = BOXES * BOX_BYTES;    // one of K or V
+    static constexpr int BOX_BYTES = 64 * 128;              // 64 rows x 128 B
+    static constexpr int TILE_BYTES = BOXES * BOX_BYTES;    // one of K or V for a unit
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-    static constexpr int SLABS = BS / 16;
 };
 
-template <int D, int BS, int STAGES>
-__global__ void __launch_bounds__(MmaCfg<D, BS, STAGES>::THREADS, 1)
+template <int D, int UPB, int STAGES>
+__global__ void __launch_bounds__(MmaCfg<D, UPB, STAGES>::THREADS, 2)
 decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __nv_bfloat16* __restrict__ q,
-                  float sl2, const uint32_t* __restrict__ bits, int nw, float* __restrict__ part,
-                  int nsplit, int max_per, int32_t* status) {
-    using Cfg = MmaCfg<D, BS, STAGES>;
-    constexpr int NCW = Cfg::NCW, G4 = 4;
+                  const __grid_constant__ CUtensorMap tmV, const DecodeArgs a) {
+    using Cfg = MmaCfg<D, UPB, STAGES>;
+    constexpr int NCW = Cfg::NCW, G4 = 4, BS = Cfg::BS;
     extern __shared__ __align__(1024) unsigned char smem_mma[];
     // carve: stages (1024-aligned) | barriers | lists | query constants
-    unsigned char* base = reinterpret_cast<unsigned char*>(
+    unsigned char* stages = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_mma) + 1023) & ~uintptr_t(1023));
-    unsigned char* stages = base;
     uint64_t* full = reinterpret_cast<uint64_t*>(stages + STAGES * Cfg::STAGE_BYTES);
     uint64_t* empty = full + STAGES;
     int32_t* blk = reinterpret_cast<int32_t*>(empty + STAGES);
-    int32_t* phys = blk + max_per;
-    uint32_t* hm = reinterpret_cast<uint32_t*>(phys + max_per);
+    int32_t* phys = blk + a.max_per;
+    uint32_t* hm = reinterpret_cast<uint32_t*>(phys + a.max_per);
     // 16-byte aligned: ml is read as float2 (max_per may be odd)
     float* qs = reinterpret_cast<float*>(
-        (reinterpret_cast<uintptr_t>(hm + max_per) + 15) & ~uintptr_t(15));   // [4][D]
+        (reinterpret_cast<uintptr_t>(hm + a.max_per) + 15) & ~uintptr_t(15));   // [4][D]
     float* aw = qs + G4 * D;                                // [4][D]
     float* ml = aw + G4 * D;                                // [D]
     float* nsl = ml + D;                                    // [4][D]
     float* dsl = nsl + G4 * D;                              // [4]
     float* cg = dsl + G4;                                   // [4]
-    __shared__ int s_nblk, s_abort;
+    __shared__ int s_nblk, s_abort, s_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv, split = blockIdx.x;
-    const int G = c.group;
+    const int G = c.group, nsplit = a.nsplit;
     int32_t L = c.lens[b];
     if (L < 0 || L > c.mbp * c.bs) L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + BS - 1) / BS;
+    const int64_t rec_base = (((int64_t)b * c.hkv + h) * nsplit + split) * G;
+    constexpr int REC = 2 * D + 4;
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -179,35 +317,31 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         s_abort = 0;
     }
     if (warp == NCW) {
-        const int n = (nb > 0) ? build_union_share(c, bits, nw, b, h, nb, split, nsplit, max_per,
-                                                   blk, phys, hm, status)
+        const int n = (nb > 0) ? build_union_share(c, a.bits, a.nw, b, h, nb, split, nsplit,
+                                                   a.max_per, blk, phys, hm, a.status)
                                : 0;
         if (lane == 0) s_nblk = n;
     } else if (nb > 0) {
-        query_setup(c, q, SPLA_BF16, b, h, qs, aw, ml, cg, tid, NCW * 32);
+        query_load(c, a.q, 1, b, h, qs, ml, tid, NCW * 32);
         asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
-        query_weights(c, b, h, qs, aw, cg, tid, NCW * 32);
+        query_max(c, b, h, qs, cg, tid);
         asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
-        const float* mrow = c.m + ((int64_t)b * c.hkv + h) * D;
-        for (int e = tid; e < G * D; e += NCW * 32) {
-            const int g = e / D, i = e % D;
-            aw[e] = expf(qs[e] + mrow[i] - cg[g]);
-        }
+        query_phi(c, b, h, qs, cg, aw, tid, NCW * 32);
     }
     __syncthreads();
     const int nblk = s_nblk;
-    const int64_t rec_base = (((int64_t)b * c.hkv + h) * nsplit + split) * G;
-    const int REC = rec_floats(D);
 
     if (nb == 0) {
         for (int e = tid; e < G * REC; e += blockDim.x) {
             const int g = e / REC, f = e % REC;
-            part[(rec_base + g) * REC + f] = (f == 0) ? -SPLA_INF : 0.f;
+            a.part[(rec_base + g) * REC + f] = (f == 0) ? -SPLA_INF : 0.f;
         }
+        finish_group<__nv_bfloat16>(c, a, b, h, reinterpret_cast<float*>(stages), tid, blockDim.x,
+                                    &s_flag);
         return;
     }
 
-    // per-lane consumer state (columns c0, c1 of the C fragments; see below)
+    // per-lane consumer state: columns c0, c1 of the 16x8 C fragments
     float m_run[2] = {-SPLA_INF, -SPLA_INF}, l_run[2] = {0.f, 0.f}, dt_run[2] = {0.f, 0.f};
     float acc[D / 16][4];
 #pragma unroll
@@ -215,53 +349,36 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     const int c0 = 2 * (lane & 3), c1 = c0 + 1;
 
     if (warp == NCW) {
-        // ---------------- producer: TMA ring
+        // ---------------- producer: TMA ring over 64-token units
         if (lane == 0) {
-            for (int it = 0; it < nblk; ++it) {
-                const int st = it % STAGES;
-                if (it >= STAGES) {
-                    if (!mbar_wait_bounded(&empty[st], ((it / STAGES) - 1) & 1)) {
-                        set_status(status, SPLA_DEV_TIMEOUT);
+            int u = 0;
+            for (int it = 0; it < nblk && !s_abort; ++it) {
+                for (int half = 0; half < UPB; ++half) {
+                    if (blk[it] * BS + half * 64 >= L) break;
+                    const int st = u % STAGES;
+                    if (u >= STAGES && !mbar_wait_bounded(&empty[st], ((u / STAGES) - 1) & 1)) {
+                        set_status(a.status, SPLA_DEV_TIMEOUT);
                         atomicExch(&s_abort, 1);
                         break;
                     }
-                }
-                if (*(volatile int*)&s_abort) break;
-                unsigned char* kst = stages + st * Cfg::STAGE_BYTES;
-                unsigned char* vst = kst + Cfg::TILE_BYTES;
-                mbar_arrive_expect_tx(&full[st], Cfg::STAGE_BYTES);
-                const int row = (phys[it] * c.hkv + h) * BS;
+                    unsigned char* kst = stages + st * Cfg::STAGE_BYTES;
+                    unsigned char* vst = kst + Cfg::TILE_BYTES;
+                    mbar_arrive_expect_tx(&full[st], Cfg::STAGE_BYTES);
+                    const int row = (phys[it] * c.hkv + h) * BS + half * 64;
 #pragma unroll
-                for (int bx = 0; bx < Cfg::BOXES; ++bx) {
-                    tma_load_2d(kst + bx * Cfg::BOX_BYTES, &tmK, &full[st], bx * 64, row);
-                    tma_load_2d(vst + bx * Cfg::BOX_BYTES, &tmV, &full[st], bx * 64, row);
+                    for (int bx = 0; bx < Cfg::BOXES; ++bx) {
+                        tma_load_2d(kst + bx * Cfg::BOX_BYTES, &tmK, &full[st], bx * 64, row);
+                        tma_load_2d(vst + bx * Cfg::BOX_BYTES, &tmV, &full[st], bx * 64, row);
+                    }
+                    ++u;
                 }
             }
         }
     } else {
         // ---------------- consumers
-        // slice of the global readout: rows [r0, r1) of S and z
-        const int r0 = (int)((int64_t)split * D / nsplit), r1 = (int)((int64_t)(split + 1) * D / nsplit);
-        const float* Sg = c.S + ((int64_t)b * c.hkv + h) * D * D;
-        const float* zg = c.z + ((int64_t)b * c.hkv + h) * D;
-        for (int j = tid; j < D; j += NCW * 32) {
-            float acc[G4] = {0.f, 0.f, 0.f, 0.f};
-            for (int i = r0; i < r1; ++i) {
-                const float sv = Sg[(int64_t)i * D + j];
-#pragma unroll
-                for (int g = 0; g < G4; ++g)
-                    if (g < G) acc[g] = fmaf(aw[g * D + i], sv, acc[g]);
-            }
-#pragma unroll
-            for (int g = 0; g < G4; ++g)
-                if (g < G) nsl[g * D + j] = acc[g];
-        }
-        if (warp < G) {
-            float s = 0.f;
-            for (int i = r0 + lane; i < r1; i += 32) s = fmaf(aw[warp * D + i], zg[i], s);
-            s = warp_sum(s);
-            if (lane == 0) dsl[warp] = s;
-        }
+        const int r0 = (int)((int64_t)split * D / nsplit);
+        const int r1 = (int)((int64_t)(split + 1) * D / nsplit);
+        state_slice(c, b, h, r0, r1, aw, nsl, dsl, tid, NCW * 32);
         // B fragments: column n = lane/4; rows k = 2*(lane%4) (+1, +8, +9) of each 16-dim step
         uint32_t qf[D / 16][2], wf[D / 16][2];
         {
@@ -285,24 +402,28 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
             }
         }
         const bool lo_half = (lane & 3) < 2;
-
-        for (int it = 0; it < nblk; ++it) {
-            const int st = it % STAGES;
-            if (!mbar_wait_bounded(&full[st], (it / STAGES) & 1)) {
-                set_status(status, SPLA_DEV_TIMEOUT);
-                atomicExch(&s_abort, 1);
-                break;
-            }
-            const unsigned char* kst = stages + st * Cfg::STAGE_BYTES;
-            unsigned char* vst = const_cast<unsigned char*>(kst) + Cfg::TILE_BYTES;
+        const int qm = lane >> 3, rr = lane & 7;
+        const int t0 = warp * 16;                       // this warp's slab of every unit
+        int u = 0;
+        bool stop = false;
+        for (int it = 0; it < nblk && !stop; ++it) {
             const int jblk = blk[it];
-            const int nvalid = min(BS, L - jblk * BS);
             const uint32_t hmask = hm[it];
-            const uint32_t kbase = smem_u32(kst), vbase = smem_u32(vst);
-            if (hmask) {
-                for (int sl = warp; sl < Cfg::SLABS; sl += NCW) {
-                    const int t0 = sl * 16;
-                    if (t0 >= nvalid) break;
+            for (int half = 0; half < UPB; ++half) {
+                const int tb = jblk * BS + half * 64;
+                if (tb >= L) break;
+                const int nvalid = min(64, L - tb);
+                const int st = u % STAGES;
+                if (!mbar_wait_bounded(&full[st], (u / STAGES) & 1)) {
+                    set_status(a.status, SPLA_DEV_TIMEOUT);
+                    atomicExch(&s_abort, 1);
+                    stop = true;
+                    break;
+                }
+                const unsigned char* kst = stages + st * Cfg::STAGE_BYTES;
+                unsigned char* vst = const_cast<unsigned char*>(kst) + Cfg::TILE_BYTES;
+                const uint32_t kbase = smem_u32(kst), vbase = smem_u32(vst);
+                if (hmask && t0 < nvalid) {
                     if (t0 + 16 > nvalid) {
                         // rows past the sequence end: zero V so that p = 0 rows add nothing
                         for (int e = lane; e < 16 * (D / 8); e += 32) {
@@ -316,7 +437,6 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
                     }
                     float cl[4] = {0.f, 0.f, 0.f, 0.f}, cw1[4] = {0.f, 0.f, 0.f, 0.f},
                           cw2[4] = {0.f, 0.f, 0.f, 0.f};
-                    const int qm = lane >> 3, rr = lane & 7;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const int t = t0 + rr + ((qm & 1) << 3);
@@ -353,8 +473,10 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
                     const bool hc1 = lo_half && c1 < G && ((hmask >> c1) & 1u);
                     const bool v00 = hc0 && tr0 < nvalid, v01 = hc1 && tr0 < nvalid;
                     const bool v10 = hc0 && tr1 < nvalid, v11 = hc1 && tr1 < nvalid;
-                    const float s00 = v00 ? cl[0] * sl2 : -SPLA_INF, s01 = v01 ? cl[1] * sl2 : -SPLA_INF;
-                    const float s10 = v10 ? cl[2] * sl2 : -SPLA_INF, s11 = v11 ? cl[3] * sl2 : -SPLA_INF;
+                    const float s00 = v00 ? cl[0] * a.sl2 : -SPLA_INF;
+                    const float s01 = v01 ? cl[1] * a.sl2 : -SPLA_INF;
+                    const float s10 = v10 ? cl[2] * a.sl2 : -SPLA_INF;
+                    const float s11 = v11 ? cl[3] * a.sl2 : -SPLA_INF;
                     const float w00 = v00 ? x[0] + y[0] : 0.f, w01 = v01 ? x[1] + y[1] : 0.f;
                     const float w10 = v10 ? x[2] + y[2] : 0.f, w11 = v11 ? x[3] + y[3] : 0.f;
                     float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
@@ -383,8 +505,9 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
                         acc[mt][3] *= g1;
                     }
                     // [P | W] as a 16 x 8 matrix in C layout: lanes with cols 4..7 take W from lane-2
-                    float wv[4] = {w00, w01, w10, w11}, pw[4];
+                    const float wv[4] = {w00, w01, w10, w11};
                     const float pv[4] = {p00, p01, p10, p11};
+                    float pw[4];
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
                         const float up = __shfl_up_sync(0xffffffffu, wv[r], 2);
@@ -405,9 +528,10 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
                         mma_bf16(acc[mt], a0, a1, a2, a3, bl0, bl1);
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+                ++u;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
         }
         // reduce the lane partials of l and D~ over the 8 lanes of each column
 #pragma unroll
@@ -420,13 +544,12 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     }
     // every consumer is done with the stage buffers once all threads pass here
     __syncthreads();
+    float* mw = reinterpret_cast<float*>(stages);           // [NCW][4]
+    float* lw = mw + NCW * 4;
+    float* dw = lw + NCW * 4;
+    float* ap = dw + NCW * 4;                               // [NCW][4][D]
+    float* an = ap + NCW * 4 * D;                           // [NCW][4][D]
     if (warp < NCW) {
-        // park per-warp results in the (now idle) stage buffers
-        float* mw = reinterpret_cast<float*>(stages);               // [NCW][4]
-        float* lw = mw + NCW * 4;
-        float* dw = lw + NCW * 4;
-        float* ap = dw + NCW * 4;                                   // [NCW][4][D]
-        float* an = ap + NCW * 4 * D;                               // [NCW][4][D]
         if (lane < 2) {
             mw[warp * 4 + c0] = m_run[0];
             mw[warp * 4 + c1] = m_run[1];
@@ -447,50 +570,40 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     }
     __syncthreads();
     // merge the consumer warps and write the partial records
-    {
-        const float* mw = reinterpret_cast<const float*>(stages);
-        const float* lw = mw + NCW * 4;
-        const float* dw = lw + NCW * 4;
-        const float* ap = dw + NCW * 4;
-        const float* an = ap + NCW * 4 * D;
-        for (int e = tid; e < G * D; e += blockDim.x) {
-            const int g = e / D, j = e % D;
-            float M = -SPLA_INF;
-            for (int w = 0; w < NCW; ++w) M = fmaxf(M, mw[w * 4 + g]);
-            float l = 0.f, o = 0.f, nt = 0.f, dt = 0.f;
-            for (int w = 0; w < NCW; ++w) {
-                const float f = (M == -SPLA_INF) ? 0.f : ex2(mw[w * 4 + g] - M);
-                l += lw[w * 4 + g] * f;
-                o += ap[(w * 4 + g) * D + j] * f;
-                nt += an[(w * 4 + g) * D + j];
-                dt += dw[w * 4 + g];
-            }
-            float* rec = part + (rec_base + g) * REC;
-            rec[4 + j] = o;
-            rec[4 + D + j] = nsl[g * D + j] - nt;
-            if (j == 0) {
-                rec[0] = M;
-                rec[1] = l;
-                rec[2] = dsl[g] - dt;
-                rec[3] = 0.f;
-            }
+    for (int e = tid; e < G * D; e += blockDim.x) {
+        const int g = e / D, j = e % D;
+        float M = -SPLA_INF;
+        for (int w = 0; w < NCW; ++w) M = fmaxf(M, mw[w * 4 + g]);
+        float l = 0.f, o = 0.f, nt = 0.f, dt = 0.f;
+        for (int w = 0; w < NCW; ++w) {
+            const float f = (M == -SPLA_INF) ? 0.f : ex2(mw[w * 4 + g] - M);
+            l += lw[w * 4 + g] * f;
+            o += ap[(w * 4 + g) * D + j] * f;
+            nt += an[(w * 4 + g) * D + j];
+            dt += dw[w * 4 + g];
+        }
+        float* rec = a.part + (rec_base + g) * REC;
+        rec[4 + j] = o;
+        rec[4 + D + j] = nsl[g * D + j] - nt;
+        if (j == 0) {
+            rec[0] = M;
+            rec[1] = l;
+            rec[2] = dsl[g] - dt;
+            rec[3] = 0.f;
         }
     }
+    // scratch for the combine lies past the merge area
+    finish_group<__nv_bfloat16>(c, a, b, h, an + NCW * 4 * D, tid, blockDim.x, &s_flag);
 }
 
 // ------------------------------------------------------------------ fp32 SIMT kernel
 // One CTA of 256 threads per (split, group). Tiles are staged through shared
 // memory as fp32; every product and sum is an fp32 FMA.
 template <typename T>
-__global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const T* __restrict__ q,
-                                                          float sl2,
-                                                          const uint32_t* __restrict__ bits,
-                                                          int nw, float* __restrict__ part,
-                                                          int nsplit, int max_per,
-                                                          int32_t* status) {
+__global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const DecodeArgs a) {
     extern __shared__ __align__(16) unsigned char smem_simt[];
     const int d = c.d, BS = c.bs, G = c.group;
-    float* Ks = reinterpret_cast<float*>(smem_simt);        // [BS][d]
+    float* Ks = reinterpret_cast<float*>(smem_simt);       // [BS][d]
     float* Vs = Ks + BS * d;                                // [BS][d]
     float* Ls = Vs + BS * d;                                // [4][BS] logits, then p
     float* Ws = Ls + 4 * BS;                                // [4][BS] phi weights
@@ -502,13 +615,14 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const T* 
     float* cg = dsl + 4;                                    // [4]
     float* fsc = cg + 4;                                    // [4] per-head rescale of this tile
     int32_t* blk = reinterpret_cast<int32_t*>(fsc + 4);
-    int32_t* phys = blk + max_per;
-    uint32_t* hm = reinterpret_cast<uint32_t*>(phys + max_per);
-    __shared__ int s_nblk;
+    int32_t* phys = blk + a.max_per;
+    uint32_t* hm = reinterpret_cast<uint32_t*>(phys + a.max_per);
+    __shared__ int s_nblk, s_flag;
     __shared__ float s_m[4], s_l[4], s_dt[4];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv, split = blockIdx.x;
+    const int nsplit = a.nsplit;
     int32_t L = c.lens[b];
     if (L < 0 || L > c.mbp * c.bs) L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + BS - 1) / BS;
@@ -517,38 +631,25 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const T* 
     if (nb == 0) {
         for (int e = tid; e < G * REC; e += blockDim.x) {
             const int g = e / REC, f = e % REC;
-            part[(rec_base + g) * REC + f] = (f == 0) ? -SPLA_INF : 0.f;
+            a.part[(rec_base + g) * REC + f] = (f == 0) ? -SPLA_INF : 0.f;
         }
+        finish_group<T>(c, a, b, h, Ks, tid, blockDim.x, &s_flag);
         return;
     }
     if (warp == 0) {
-        const int n = build_union_share(c, bits, nw, b, h, nb, split, nsplit, max_per, blk, phys,
-                                        hm, status);
+        const int n = build_union_share(c, a.bits, a.nw, b, h, nb, split, nsplit, a.max_per, blk,
+                                        phys, hm, a.status);
         if (lane == 0) s_nblk = n;
     }
-    query_setup(c, q, sizeof(T) == 2 ? SPLA_BF16 : SPLA_F32, b, h, qs, aw, ml, cg, tid, blockDim.x);
+    query_load(c, a.q, sizeof(T) == 2, b, h, qs, ml, tid, blockDim.x);
     __syncthreads();
-    query_weights(c, b, h, qs, aw, cg, tid, blockDim.x);
+    query_max(c, b, h, qs, cg, tid);
     __syncthreads();
-    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
-    for (int e = tid; e < G * d; e += blockDim.x) aw[e] = expf(qs[e] + mrow[e % d] - cg[e / d]);
+    query_phi(c, b, h, qs, cg, aw, tid, blockDim.x);
     if (tid < 4) { s_m[tid] = -SPLA_INF; s_l[tid] = 0.f; s_dt[tid] = 0.f; }
     __syncthreads();
     const int r0 = (int)((int64_t)split * d / nsplit), r1 = (int)((int64_t)(split + 1) * d / nsplit);
-    const float* Sg = c.S + ((int64_t)b * c.hkv + h) * d * d;
-    const float* zg = c.z + ((int64_t)b * c.hkv + h) * d;
-    for (int e = tid; e < G * d; e += blockDim.x) {
-        const int g = e / d, j = e % d;
-        float s = 0.f;
-        for (int i = r0; i < r1; ++i) s = fmaf(aw[g * d + i], Sg[(int64_t)i * d + j], s);
-        nsl[e] = s;
-    }
-    if (warp < G) {
-        float s = 0.f;
-        for (int i = r0 + lane; i < r1; i += 32) s = fmaf(aw[warp * d + i], zg[i], s);
-        s = warp_sum(s);
-        if (lane == 0) dsl[warp] = s;
-    }
+    state_slice(c, b, h, r0, r1, aw, nsl, dsl, tid, blockDim.x);
     const int nblk = s_nblk;
     // accumulators: thread owns (g, j) pairs e = tid + 256*u
     constexpr int PU = 2;                                   // G*d <= 512
@@ -573,12 +674,12 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const T* 
             if (g < G && t < nvalid && ((hmask >> g) & 1u)) {
                 float sacc = 0.f, wacc = 0.f;
                 for (int u = 0; u < d; ++u) {
-                    const int i = (u + t) % d;
+                    const int i = (u + t) & (d - 1);
                     const float kv = Ks[t * d + i];
                     sacc = fmaf(qs[g * d + i], kv, sacc);
                     wacc = fmaf(aw[g * d + i], ex2(fmaf(kv, SPLA_LOG2E, -ml[i])), wacc);
                 }
-                lg = sacc * sl2;
+                lg = sacc * a.sl2;
                 w = wacc;
             }
             Ls[e] = lg;
@@ -616,13 +717,13 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const T* 
             const int e = tid + 256 * u;
             if (e < G * d) {
                 const int g = e / d, j = e % d;
-                float a = acc[u] * fsc[g], n = ntl[u];
+                float av = acc[u] * fsc[g], n = ntl[u];
                 for (int t = 0; t < nvalid; ++t) {
                     const float vv = Vs[t * d + j];
-                    a = fmaf(Ls[g * BS + t], vv, a);
+                    av = fmaf(Ls[g * BS + t], vv, av);
                     n = fmaf(Ws[g * BS + t], vv, n);
                 }
-                acc[u] = a;
+                acc[u] = av;
                 ntl[u] = n;
             }
         }
@@ -633,7 +734,7 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const T* 
         const int e = tid + 256 * u;
         if (e < G * d) {
             const int g = e / d, j = e % d;
-            float* rec = part + (rec_base + g) * REC;
+            float* rec = a.part + (rec_base + g) * REC;
             rec[4 + j] = acc[u];
             rec[4 + d + j] = nsl[e] - ntl[u];
             if (j == 0) {
@@ -644,144 +745,75 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const T* 
             }
         }
     }
-}
-
-// ------------------------------------------------------------------ combine
-template <typename T>
-__global__ void __launch_bounds__(128) combine_kernel(CacheView c, const float* __restrict__ part,
-                                                      int nsplit, const int32_t* __restrict__ nsel,
-                                                      const float* __restrict__ gamma, float eps,
-                                                      int no_rla, T* __restrict__ out,
-                                                      float* __restrict__ o_sp,
-                                                      float* __restrict__ o_rl) {
-    const int d = c.d, G = c.group;
-    const int b = blockIdx.x / c.hq, hq = blockIdx.x % c.hq;
-    const int h = hq / G, g = hq % G;
-    const int REC = rec_floats(d);
-    __shared__ float red[4];
-    int32_t L = c.lens[b];
-    L = max(0, min(L, c.mbp * c.bs));
-    const int nb = (L + c.bs - 1) / c.bs;
-    const bool all_sel = nsel[(int64_t)b * c.hq + hq] >= nb;
-    const float* recs = part + (((int64_t)b * c.hkv + h) * nsplit * G) * REC;
-    auto rec = [&](int s) { return recs + ((int64_t)s * G + g) * REC; };
-    float M = -SPLA_INF;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, rec(s)[0]);
-    float Dr = 0.f;
-    float lsum = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-        const float* r = rec(s);
-        lsum += (M == -SPLA_INF) ? 0.f : r[1] * ex2(r[0] - M);
-        Dr += r[2];
-    }
-    const bool rla_off = no_rla || all_sel || !(Dr > 0.f) || L == 0;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        float o = 0.f, R = 0.f;
-        for (int s = 0; s < nsplit; ++s) {
-            const float* r = rec(s);
-            if (M != -SPLA_INF) o += r[4 + j] * ex2(r[0] - M);
-            R += r[4 + d + j];
-        }
-        o = (lsum > 0.f) ? o / lsum : 0.f;
-        const float rl = rla_off ? 0.f : R / Dr;
-        // RMS over d
-        float sq = rl * rl;
-        sq = warp_sum(sq);
-        if (d > 32) {
-            if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
-            __syncthreads();
-            sq = 0.f;
-            for (int w = 0; w < (min((int)blockDim.x, d) + 31) / 32; ++w) sq += red[w];
-            __syncthreads();
-        }
-        const float inv = rsqrtf(sq / d + eps);
-        const float gm = gamma ? gamma[(int64_t)hq * d + j] : 1.f;
-        const int64_t oi = ((int64_t)b * c.hq + hq) * d + j;
-        out[oi] = from_f<T>(o + gm * rl * inv);
-        if (o_sp) o_sp[oi] = o;
-        if (o_rl) o_rl[oi] = rl;
-    }
+    __syncthreads();
+    finish_group<T>(c, a, b, h, Ks, tid, blockDim.x, &s_flag);
 }
 
 // ------------------------------------------------------------------ host launchers
-template <int D, int BS, int STAGES>
+template <int D, int UPB, int STAGES>
 static size_t mma_smem_bytes(int max_per) {
-    using Cfg = MmaCfg<D, BS, STAGES>;
+    using Cfg = MmaCfg<D, UPB, STAGES>;
     return 1024 + (size_t)STAGES * Cfg::STAGE_BYTES + 2 * STAGES * sizeof(uint64_t) +
            3 * (size_t)max_per * 4 + 16 + (size_t)(4 * D * 2 + D + 4 * D + 8) * 4 + 64;
 }
 
-template <int D, int BS, int STAGES>
+template <int D, int UPB, int STAGES>
 static cudaError_t launch_mma_t(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
-                                const void* q, float sl2, const uint32_t* bits, int nw,
-                                float* part, int nsplit, int max_per, int32_t* status,
-                                cudaStream_t s) {
-    using Cfg = MmaCfg<D, BS, STAGES>;
-    const size_t smem = mma_smem_bytes<D, BS, STAGES>(max_per);
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D, BS, STAGES>,
+                                const DecodeArgs& a, cudaStream_t s) {
+    using Cfg = MmaCfg<D, UPB, STAGES>;
+    const size_t smem = mma_smem_bytes<D, UPB, STAGES>(a.max_per);
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D, UPB, STAGES>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(nsplit, c.batch * c.hkv);
-    decode_mma_kernel<D, BS, STAGES><<<grid, Cfg::THREADS, smem, s>>>(
-        c, tk, tv, (const __nv_bfloat16*)q, sl2, bits, nw, part, nsplit, max_per, status);
+    dim3 grid(a.nsplit, c.batch * c.hkv);
+    decode_mma_kernel<D, UPB, STAGES><<<grid, Cfg::THREADS, smem, s>>>(c, tk, tv, a);
     return cudaGetLastError();
 }
 
+// The merge area plus the combine scratch reuse the stage ring; they must fit
+// (nsplit is at most kMaxSplit, see the host layout).
+constexpr int kMaxSplit = 512;
+static_assert(3 * MmaCfg<128, 1, 3>::STAGE_BYTES >=
+                  (2 * 4 * 4 * 128 + 48 + 32 + 4 * kMaxSplit + 8 * 128) * 4,
+              "stage ring too small for the merge and combine scratch");
+static_assert(4 * MmaCfg<64, 1, 4>::STAGE_BYTES >=
+                  (2 * 4 * 4 * 64 + 48 + 32 + 4 * kMaxSplit + 8 * 64) * 4,
+              "stage ring too small for the merge and combine scratch");
+
 size_t mma_smem_for(int d, int bs, int max_per) {
-    if (d == 128 && bs == 64) return mma_smem_bytes<128, 64, 4>(max_per);
-    if (d == 128 && bs == 128) return mma_smem_bytes<128, 128, 3>(max_per);
-    if (d == 64 && bs == 64) return mma_smem_bytes<64, 64, 4>(max_per);
-    return mma_smem_bytes<64, 128, 4>(max_per);
+    if (d == 128) return bs == 64 ? mma_smem_bytes<128, 1, 3>(max_per) : mma_smem_bytes<128, 2, 3>(max_per);
+    return bs == 64 ? mma_smem_bytes<64, 1, 4>(max_per) : mma_smem_bytes<64, 2, 4>(max_per);
 }
 
 cudaError_t launch_decode_mma(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
-                              const void* q, float sl2, const uint32_t* bits, int nw, float* part,
-                              int nsplit, int max_per, int32_t* status, cudaStream_t s) {
-    if (c.d == 128 && c.bs == 64)
-        return launch_mma_t<128, 64, 4>(c, tk, tv, q, sl2, bits, nw, part, nsplit, max_per, status, s);
-    if (c.d == 128 && c.bs == 128)
-        return launch_mma_t<128, 128, 3>(c, tk, tv, q, sl2, bits, nw, part, nsplit, max_per, status, s);
-    if (c.d == 64 && c.bs == 64)
-        return launch_mma_t<64, 64, 4>(c, tk, tv, q, sl2, bits, nw, part, nsplit, max_per, status, s);
-    return launch_mma_t<64, 128, 4>(c, tk, tv, q, sl2, bits, nw, part, nsplit, max_per, status, s);
+                              const DecodeArgs& a, cudaStream_t s) {
+    if (c.d == 128 && c.bs == 64) return launch_mma_t<128, 1, 3>(c, tk, tv, a, s);
+    if (c.d == 128 && c.bs == 128) return launch_mma_t<128, 2, 3>(c, tk, tv, a, s);
+    if (c.d == 64 && c.bs == 64) return launch_mma_t<64, 1, 4>(c, tk, tv, a, s);
+    return launch_mma_t<64, 2, 4>(c, tk, tv, a, s);
 }
 
 size_t simt_smem_for(int d, int bs, int max_per) {
-    return (size_t)(2 * bs * d + 8 * bs + 4 * d * 3 + d + 16) * 4 + 3 * (size_t)max_per * 4 + 64;
+    const size_t tiles = (size_t)(2 * bs * d + 8 * bs + 4 * d * 3 + d + 16) * 4;
+    const size_t comb = (size_t)(48 + 32 + 4 * kMaxSplit + 8 * d) * 4;   // combine scratch in Ks
+    return (tiles > comb ? tiles : comb) + 3 * (size_t)max_per * 4 + 64;
 }
 
-cudaError_t launch_decode_simt(const CacheView& c, int dtype, const void* q, float sl2,
-                               const uint32_t* bits, int nw, float* part, int nsplit, int max_per,
-                               int32_t* status, cudaStream_t s) {
-    const size_t smem = simt_smem_for(c.d, c.bs, max_per);
-    dim3 grid(nsplit, c.batch * c.hkv);
+cudaError_t launch_decode_simt(const CacheView& c, int dtype, const DecodeArgs& a, cudaStream_t s) {
+    const size_t smem = simt_smem_for(c.d, c.bs, a.max_per);
+    dim3 grid(a.nsplit, c.batch * c.hkv);
     cudaError_t e;
     if (dtype == SPLA_BF16) {
         e = cudaFuncSetAttribute(decode_simt_kernel<__nv_bfloat16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_simt_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(
-            c, (const __nv_bfloat16*)q, sl2, bits, nw, part, nsplit, max_per, status);
+        decode_simt_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(c, a);
     } else {
         e = cudaFuncSetAttribute(decode_simt_kernel<float>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_simt_kernel<float><<<grid, 256, smem, s>>>(c, (const float*)q, sl2, bits, nw, part,
-                                                          nsplit, max_per, status);
+        decode_simt_kernel<float><<<grid, 256, smem, s>>>(c, a);
     }
-    return cudaGetLastError();
-}
-
-cudaError_t launch_combine(const CacheView& c, int dtype, const float* part, int nsplit,
-                           const int32_t* nsel, const float* gamma, float eps, int no_rla,
-                           void* out, float* o_sp, float* o_rl, cudaStream_t s) {
-    const int threads = c.d;                                 // 64 or 128
-    if (dtype == SPLA_BF16)
-        combine_kernel<__nv_bfloat16><<<c.batch * c.hq, threads, 0, s>>>(
-            c, part, nsplit, nsel, gamma, eps, no_rla, (__nv_bfloat16*)out, o_sp, o_rl);
-    else
-        combine_kernel<float><<<c.batch * c.hq, threads, 0, s>>>(c, part, nsplit, nsel, gamma, eps,
-                                                                 no_rla, (float*)out, o_sp, o_rl);
     return cudaGetLastError();
 }
 

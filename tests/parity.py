@@ -74,7 +74,13 @@ def compare_head(gpu: dict, oc: so.OracleCache, q, gamma, b, hq, dtype: str) -> 
     gsel = [int(x) for x in gpu["sel"] if x >= 0]
     fref = so.decode_head(np.asarray(q[b, hq], np.float64), g, p, gamma[hq], forced_sel=gsel)
     tol = TOL[dtype]
-    k = kappa(q[b, hq], g, p, gsel) if not p.no_rla else 1.0
+    all_kept = len(gsel) == fref["n_blocks"]
+    if all_kept or p.no_rla:
+        # nothing left for the residual: exactly zero on both sides
+        assert np.all(np.asarray(gpu["o_rla"]) == 0) and np.all(fref["o_rla"] == 0)
+        k = 1.0
+    else:
+        k = kappa(q[b, hq], g, p, gsel)
 
     def err(name):
         r = fref[name]

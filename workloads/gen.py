@@ -147,11 +147,11 @@ def get(name: str, **overrides) -> Workload:
     return w
 
 
-def scaled(name: str, context_lens, **overrides) -> Workload:
+def scaled(base: str, context_lens, **overrides) -> Workload:
     """The named workload's structure (heads, d, block, top-k, distributions) at other lengths."""
     lens = tuple(int(x) for x in context_lens)
-    overrides.setdefault("name", f"{name}-small")
-    return replace(CONFIGS[name], context_lens=lens, batch=len(lens), **overrides)
+    overrides.setdefault("name", f"{base}-small")
+    return replace(CONFIGS[base], context_lens=lens, batch=len(lens), **overrides)
 
 
 # --------------------------------------------------------------------------- rng helpers
