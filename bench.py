@@ -178,12 +178,13 @@ def run_ours(args):
     out = torch.empty((w.batch, w.num_q_heads, w.head_dim), dtype=steps[0][2].dtype, device=dev)
     sels = torch.empty((2 * K, w.batch, w.num_q_heads, w.top_k + w.n_sink + w.n_local),
                        dtype=torch.int32, device=dev)
-    lens_after = []
     flush = L2Flush(dev)
+
+    ones = torch.ones((w.batch,), dtype=torch.int32, device=dev)    # one new token per sequence
 
     def step(s, sel=None):
         k, v, q = steps[s]
-        cache.append(k, v)
+        cache.append(k, v, ones)
         cache.decode(q, gamma, out, sel)
 
     for s in range(W):
@@ -237,7 +238,7 @@ def run_ours(args):
     # ---- e2e: host buffers through the same calls, copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        e2e = e2e_pass(w, cache, steps, W + 2 * K, K, gamma, flush, dev, stream)
+        e2e = e2e_pass(w, cache, steps, W + 2 * K, K, gamma, flush, dev, stream, ones)
 
     # ---- reduce over ranks
     t_max = t_total
@@ -290,7 +291,7 @@ def run_ours(args):
             "kernels_ms": {n: round(float(np.mean(kt[:, j])), 5) for j, n in enumerate(kernel_names)},
             "kernel_share": {n: round(float(share[j]), 4) for j, n in enumerate(kernel_names)},
             "clocks": clk.summary(),
-            "gpu_launches": 7 * K,
+            "gpu_launches": 6 * K,
             "dev_status": status,
         }
         if e2e is not None:
@@ -305,7 +306,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def e2e_pass(w, cache, steps, s0, K, gamma, flush, dev, stream):
+def e2e_pass(w, cache, steps, s0, K, gamma, flush, dev, stream, ones):
     """Per step: pinned host -> device copy of (k, v, q), append + decode, device -> host of out."""
     import torch
     from workloads import gen
@@ -330,7 +331,7 @@ def e2e_pass(w, cache, steps, s0, K, gamma, flush, dev, stream):
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         dq.copy_(hq, non_blocking=True)
-        cache.append(dk, dv)
+        cache.append(dk, dv, ones)
         cache.decode(dq, gamma, out)
         hout.copy_(out, non_blocking=True)
         e1[i].record(stream)

@@ -66,7 +66,8 @@ class SplaDecodeCache:
         self.num_phys_blocks = int(num_phys_blocks)
         self.k_pool = torch.empty((num_phys_blocks, Hkv, B, d), dtype=cfg.torch_dtype, device=dev)
         self.v_pool = torch.empty_like(self.k_pool)
-        self.blk_stats = torch.zeros((num_phys_blocks, Hkv, 2, d), dtype=torch.float32, device=dev)
+        self.blk_stats = torch.zeros((batch, Hkv, self.max_blocks_per_seq, 2, d),
+                                     dtype=torch.float32, device=dev)
         self.S = torch.empty((batch, Hkv, d, d), dtype=torch.float32, device=dev)
         self.z = torch.empty((batch, Hkv, d), dtype=torch.float32, device=dev)
         self.m = torch.empty((batch, Hkv, d), dtype=torch.float32, device=dev)

@@ -12,21 +12,22 @@ cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s);
 cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, const void* v_new,
                           const int32_t* n_new, int32_t max_new, int32_t* status, cudaStream_t s);
 cudaError_t launch_score(const CacheView& c, int dtype, const void* q, double scale,
-                         int first_order, float* scores, int chunk, int32_t* status,
-                         cudaStream_t s);
+                         int first_order, float* scores, int chunk, float* gread,
+                         int32_t* status, cudaStream_t s);
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
                           const float* scores, uint32_t* bits, int nw, int32_t* nsel,
-                          int32_t* sel_idx, int kcap, int32_t* counters, cudaStream_t s);
+                          int32_t* sel_idx, int kcap, cudaStream_t s);
 cudaError_t launch_decode_mma(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
                               const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_simt(const CacheView& c, int dtype, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_combine(const CacheView& c, int dtype, const DecodeArgs& a, cudaStream_t s);
 size_t mma_smem_for(int d, int bs, int max_per);
 size_t simt_smem_for(int d, int bs, int max_per);
 
-// The split heuristic is tuned for the 148-SM B200 (two decode CTAs per SM);
+// The split heuristic is tuned for the 148-SM B200 (three decode CTAs per SM);
 // results do not depend on it.
 constexpr int kTargetCtas = 148;
-constexpr int kDecodeSlots = 2 * kTargetCtas;
+constexpr int kDecodeSlots = 3 * kTargetCtas;
 constexpr int kMaxSplit = 512;
 constexpr int kMaxSmem = 227 * 1024;
 
@@ -104,10 +105,10 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     ns = std::max(1, std::min(ns, std::min(kMaxSplit, std::max(1, umax / 2))));
     L.nsplit = ns;
     L.max_per = (umax + ns - 1) / ns + 1;
-    // scoring chunk: 128 blocks per CTA (one pass of its 4 warps); smaller if that
-    // leaves fewer than four CTAs per SM
-    int chunk = 128;
-    while (chunk > 32 && (int64_t)groups * ((mbp + chunk - 1) / chunk) < 4 * kTargetCtas) chunk >>= 1;
+    // scoring chunk: 256 blocks per CTA; smaller while that leaves fewer than two
+    // CTAs per SM
+    int chunk = 256;
+    while (chunk > 32 && (int64_t)groups * ((mbp + chunk - 1) / chunk) < 2 * kTargetCtas) chunk >>= 1;
     L.score_chunk = chunk;
     size_t off = 0;
     L.off_scores = off;
@@ -118,8 +119,8 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     off = align256(off + (size_t)batch * p->num_q_heads * sizeof(int32_t));
     L.off_part = off;
     off = align256(off + (size_t)groups * ns * G * L.rec * sizeof(float));
-    L.off_cnt = off;
-    off = align256(off + (size_t)groups * sizeof(int32_t));
+    L.off_gread = off;
+    off = align256(off + (size_t)groups * G * (p->head_dim + 4) * sizeof(float));
     L.total = off;
     return L;
 }
@@ -255,13 +256,13 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     const int no_rla = (params->flags & SPLA_FLAG_NO_RLA) ? 1 : 0;
 
     prof_mark(0, s);
+    float* gread = reinterpret_cast<float*>(ws + L.off_gread);
     cudaError_t e = launch_score(v, params->dtype, q, scale, first_order, scores, L.score_chunk,
-                                 dev_status, s);
+                                 gread, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(1, s);
-    int32_t* counters = reinterpret_cast<int32_t*>(ws + L.off_cnt);
     e = launch_select(v, params->top_k, params->n_sink, params->n_local, scores, bits, L.nw, nsel,
-                      sel_idx, L.kcap, counters, s);
+                      sel_idx, L.kcap, s);
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(2, s);
     DecodeArgs da;
@@ -273,7 +274,7 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     da.bits = bits;
     da.nsel = nsel;
     da.part = part;
-    da.counters = counters;
+    da.gread = gread;
     da.status = dev_status;
     da.nw = L.nw;
     da.nsplit = L.nsplit;
@@ -291,6 +292,8 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     }
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(3, s);
+    e = launch_combine(v, params->dtype, da, s);
+    if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(4, s);
     return SPLA_OK;
 }

@@ -36,6 +36,8 @@ __global__ void __launch_bounds__(256) append_kv_stats_kernel(CacheView c, const
                                                               int32_t max_new, int32_t* status) {
     const int b = blockIdx.y / c.hkv;
     const int h = blockIdx.y % c.hkv;
+    pdl_trigger();
+    pdl_wait();
     int32_t L0, n;
     if (!append_ok(c, n_new, max_new, b, &L0, &n)) {
         if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0)
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(256) append_kv_stats_kernel(CacheView c, const
     const int nj = t_end - (int)blk_lo;
     for (int e = threadIdx.x; e < nj * d; e += blockDim.x) ktile[e] = to_f(kp[e]);
     __syncthreads();
-    float* st = c.stats + ((int64_t)phys * c.hkv + h) * 2 * d;
+    float* st = c.stats + (((int64_t)b * c.hkv + h) * c.mbp + lb) * 2 * d;
     const int parts = blockDim.x / d;                // threads per dimension (2 at d=128, 4 at 64)
     const int i = threadIdx.x % d, part = threadIdx.x / d;
     __shared__ double red[256];
@@ -106,6 +108,8 @@ __global__ void __launch_bounds__(256) append_state_kernel(CacheView c, const T*
                                                            int32_t max_new) {
     const int b = blockIdx.y / c.hkv;
     const int h = blockIdx.y % c.hkv;
+    pdl_trigger();
+    pdl_wait();
     int32_t L0, n;
     if (!append_ok(c, n_new, max_new, b, &L0, &n) || n == 0) return;
     const int d = c.d;
@@ -162,6 +166,8 @@ __global__ void __launch_bounds__(256) append_state_kernel(CacheView c, const T*
 }
 
 __global__ void append_advance_kernel(CacheView c, const int32_t* n_new, int32_t max_new) {
+    pdl_trigger();
+    pdl_wait();
     for (int b = threadIdx.x; b < c.batch; b += blockDim.x) {
         int32_t L0, n;
         if (append_ok(c, n_new, max_new, b, &L0, &n)) c.lens[b] = L0 + n;
@@ -203,21 +209,24 @@ cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, cons
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
         }
+        cudaError_t e;
         if (dtype == SPLA_BF16) {
-            append_kv_stats_kernel<__nv_bfloat16><<<g1, 256, smem, s>>>(
-                c, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_new, max_new, status);
-            append_state_kernel<__nv_bfloat16><<<g2, 256, 0, s>>>(
-                c, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_new, max_new);
+            using B16 = __nv_bfloat16;
+            e = launch_pdl(append_kv_stats_kernel<B16>, g1, dim3(256), smem, s, c,
+                           (const B16*)k_new, (const B16*)v_new, n_new, max_new, status);
+            if (e == cudaSuccess)
+                e = launch_pdl(append_state_kernel<B16>, g2, dim3(256), 0, s, c, (const B16*)k_new,
+                               (const B16*)v_new, n_new, max_new);
         } else {
-            append_kv_stats_kernel<float><<<g1, 256, smem, s>>>(c, (const float*)k_new,
-                                                            (const float*)v_new, n_new, max_new,
-                                                            status);
-            append_state_kernel<float><<<g2, 256, 0, s>>>(c, (const float*)k_new,
-                                                         (const float*)v_new, n_new, max_new);
+            e = launch_pdl(append_kv_stats_kernel<float>, g1, dim3(256), smem, s, c,
+                           (const float*)k_new, (const float*)v_new, n_new, max_new, status);
+            if (e == cudaSuccess)
+                e = launch_pdl(append_state_kernel<float>, g2, dim3(256), 0, s, c,
+                               (const float*)k_new, (const float*)v_new, n_new, max_new);
         }
+        if (e != cudaSuccess) return e;
     }
-    append_advance_kernel<<<1, 128, 0, s>>>(c, n_new, max_new);
-    return cudaGetLastError();
+    return launch_pdl(append_advance_kernel, dim3(1), dim3(128), 0, s, c, n_new, max_new);
 }
 
 }  // namespace spla

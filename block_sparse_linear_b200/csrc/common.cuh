@@ -6,7 +6,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/spla.h"
+#include "spla.h"
 
 #define SPLA_INF __int_as_float(0x7f800000)
 #define SPLA_LOG2E 1.4426950408889634f
@@ -18,7 +18,7 @@ namespace spla {
 struct CacheView {
     const void* k_pool;
     const void* v_pool;
-    float* stats;            // [phys][Hkv][2][d]
+    float* stats;            // [batch][Hkv][mbp][2][d], logical block order
     float* S;                // [batch][Hkv][d][d]
     float* z;                // [batch][Hkv][d]
     float* m;                // [batch][Hkv][d]
@@ -36,7 +36,7 @@ struct DecodeLayout {
     int32_t rec;             // floats per partial record
     int32_t score_chunk;     // blocks per scoring CTA
     int32_t max_per;         // union blocks one decode CTA may receive
-    size_t off_scores, off_bits, off_nsel, off_part, off_cnt, total;
+    size_t off_scores, off_bits, off_nsel, off_part, off_gread, total;
 };
 
 // Per-call arguments of the decode kernels beyond the cache.
@@ -49,7 +49,7 @@ struct DecodeArgs {
     const uint32_t* bits;       // [batch][Hq][nw] selection bitsets
     const int32_t* nsel;        // [batch][Hq]
     float* part;                // [batch*Hkv][nsplit][G][rec]
-    int32_t* counters;          // [batch*Hkv], zeroed by the selection kernel
+    const float* gread;         // [batch*Hkv][G][d+4]: global readout N (d), then D
     int32_t* status;
     int nw, nsplit, max_per, no_rla;
     float sl2, eps;
@@ -57,7 +57,8 @@ struct DecodeArgs {
 
 // Partial record of one decode CTA for one query head:
 //   [0] m (running max, log2 units), [1] l (softmax denominator),
-//   [2] Dr = D_slice - D~_part, [3] unused, [4..4+d) acc, [4+d..4+2d) R = N_slice - N~_part
+//   [2] D~_part, [3] unused, [4..4+d) acc, [4+d..4+2d) N~_part
+// (the kept blocks' linear-attention numerator and denominator over this CTA's share)
 __host__ __device__ inline int rec_floats(int d) { return 2 * d + 4; }
 
 // ------------------------------------------------------------------ small math
@@ -102,6 +103,14 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ void set_status(int32_t* st, int32_t bits) {
     if (st) atomicOr(st, bits);
 }
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel after the first of a call is launched with programmatic stream
+// serialisation: it may start while its predecessor drains, and waits here
+// before touching anything the predecessor (or an earlier kernel) wrote.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel in the stream launch once every CTA of this grid has run this.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ------------------------------------------------------------------ mbarrier / TMA (no multicast)
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -156,6 +165,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_
         :: "r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y) : "memory");
 }
 
+// 1-D bulk copy global -> this CTA's shared memory (16-byte aligned, size a
+// multiple of 16), completing on `bar`. No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
 // ------------------------------------------------------------------ warp-level MMA plumbing
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
@@ -187,5 +204,24 @@ __device__ __forceinline__ void mma_bf16(float* c, uint32_t a0, uint32_t a1, uin
 __device__ __forceinline__ uint32_t swz128(int row, int chunk) {
     return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
+
+#ifdef __CUDACC__
+// Host: launch `kern` with programmatic stream serialisation.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+#endif
 
 }  // namespace spla

@@ -12,21 +12,21 @@
 //   * forms the union of the G heads' selections from their bitsets and takes
 //     an equal share of it (a union block is read once for all G heads; a head
 //     that did not select it is masked out of it);
-//   * reads rows [s*d/nsplit, (s+1)*d/nsplit) of the state S, z and computes
-//     that slice of the global linear-attention readout N, D;
 //   * streams its blocks' K and V tiles and accumulates, per head, the online
 //     softmax (m, l, acc = sum p v) and the kept blocks' linear-attention
 //     numerator and denominator (N~ = sum w v, D~ = sum w) with
 //     w_t = sum_i exp(q_i + m_i - c) exp(k_t,i - m_i);
-//   * writes one partial record per head: m, l, acc, R = N_slice - N~, Dr = D_slice - D~.
-// The last CTA of a group to finish (an atomic counter) merges the group's
-// records: log-sum-exp merge of the softmax partials, o_rla = sum R / sum Dr,
-// RMSNorm, out = o_sparse + gamma * RMSNorm(o_rla).
+//   * writes one partial record per head: m, l, acc, N~, D~.
+// combine_kernel (one CTA per group, launched right behind) merges the group's
+// records: log-sum-exp merge of the softmax partials, o_rla = (N - N~)/(D - D~)
+// with the global readout N, D the scoring kernel computed from S, z;
+// RMSNorm; out = o_sparse + gamma * RMSNorm(o_rla).
 //
-// decode_mma_kernel (bf16 K/V): 4 consumer warps + 1 TMA producer warp, two
-// CTAs per SM. The pipeline unit is a 64-token tile of one (block, KV head):
-// its K and V come by 2-D tiled TMA (128-byte swizzle, no multicast) into a
-// 3-deep mbarrier ring (a 128-token block is two units). Each consumer warp
+// decode_mma_kernel (bf16 K/V): 4 consumer warps + 1 TMA producer warp, three
+// CTAs per SM (128 registers). The pipeline unit is a 64-token tile of one
+// (block, KV head): its K and V come by 2-D tiled TMA (128-byte swizzle, no
+// multicast) into a 2-deep mbarrier ring per CTA, so six units per SM are in
+// flight (a 128-token block is two units). Each consumer warp
 // owns one 16-token slab of a unit and runs the G-head contractions on tensor
 // cores (mma.sync m16n8k16 bf16, fp32 accumulate):
 //   logits  = K(16 x d) . Q^T(d x 8)            (q exact in bf16)
@@ -39,63 +39,82 @@
 namespace spla {
 
 // ------------------------------------------------------------------ shared prologue pieces
-// Union of the G heads' selections for this CTA's share (run by one warp).
-// Writes blk[], phys[], hm[] for union positions [u0, u1) and returns u1 - u0.
+// Union of the G heads' selections, this CTA's share, built by all nthr threads:
+// per-word union popcounts, one warp's exclusive scan, parallel extraction of
+// the share's blocks and head masks, then parallel block-table lookups.
+// wcnt: >= nw ints of scratch. Returns the share's length (all threads).
 __device__ int build_union_share(const CacheView& c, const uint32_t* bits, int nw, int b, int h,
                                  int nb, int split, int nsplit, int max_per, int32_t* blk,
-                                 int32_t* phys, uint32_t* hm, int32_t* status) {
-    const int lane = threadIdx.x & 31;
+                                 int32_t* phys, uint32_t* hm, int* wcnt, int* s_n,
+                                 int32_t* status, int tid, int nthr) {
+    const int lane = tid & 31, warp = tid >> 5;
     const int G = c.group;
     const int nwu = (nb + 31) >> 5;
-    const int wpl = (nwu + 31) >> 5;
     const uint32_t* hb = bits + ((int64_t)b * c.hq + h * G) * nw;
     auto word = [&](int w) -> uint32_t {
         uint32_t u = 0u;
-        for (int g = 0; g < G; ++g) u |= hb[(int64_t)g * nw + w];
+        for (int g = 0; g < G; ++g) u |= __ldg(hb + (int64_t)g * nw + w);
         if (w == nwu - 1 && (nb & 31)) u &= (1u << (nb & 31)) - 1u;
         return u;
     };
-    const int w0 = lane * wpl, w1 = min(nwu, w0 + wpl);
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(word(w));
-    int x = cnt;
+    for (int w = tid; w < nwu; w += nthr) wcnt[w] = __popc(word(w));
+    __syncthreads();
+    if (warp == 0) {
+        const int wpl = (nwu + 31) >> 5;
+        const int w0 = lane * wpl, w1 = min(nwu, w0 + wpl);
+        int cnt = 0;
+        for (int w = w0; w < w1; ++w) cnt += wcnt[w];
+        int x = cnt;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        int run = x - cnt;
+        for (int w = w0; w < w1; ++w) {
+            const int v = wcnt[w];
+            wcnt[w] = run;
+            run += v;
+        }
+        if (lane == 31) {
+            const int U = x;
+            s_n[0] = (int)(((int64_t)split * U) / nsplit);          // u0
+            s_n[1] = (int)(((int64_t)(split + 1) * U) / nsplit);    // u1
+        }
     }
-    const int U = __shfl_sync(0xffffffffu, x, 31);
-    const int u0 = (int)(((int64_t)split * U) / nsplit);
-    const int u1 = (int)(((int64_t)(split + 1) * U) / nsplit);
-    int r = x - cnt;
-    for (int w = w0; w < w1 && r < u1; ++w) {
+    __syncthreads();
+    const int u0 = s_n[0], u1 = s_n[1];
+    for (int w = tid; w < nwu; w += nthr) {
+        const int base = wcnt[w];
+        if (base >= u1) continue;
         uint32_t u = word(w);
-        const int pc = __popc(u);
-        if (r + pc <= u0) { r += pc; continue; }
+        if (base + __popc(u) <= u0) continue;
+        int r = base;
         while (u) {
             const int bit = __ffs(u) - 1;
             u &= u - 1u;
-            if (r >= u0 && r < u1) {
-                const int idx = r - u0;
-                const int j = (w << 5) + bit;
+            if (r >= u0 && r < u1 && r - u0 < max_per) {
                 uint32_t mask = 0u;
-                for (int g = 0; g < G; ++g) mask |= ((hb[(int64_t)g * nw + w] >> bit) & 1u) << g;
-                int32_t p = c.table[(int64_t)b * c.mbp + j];
-                if (p < 0 || p >= c.num_phys) {
-                    set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
-                    p = 0;
-                    mask = 0u;
-                }
-                if (idx < max_per) {
-                    blk[idx] = j;
-                    phys[idx] = p;
-                    hm[idx] = mask;
-                }
+                for (int g = 0; g < G; ++g) mask |= ((__ldg(hb + (int64_t)g * nw + w) >> bit) & 1u) << g;
+                blk[r - u0] = (w << 5) + bit;
+                hm[r - u0] = mask;
             }
             ++r;
         }
     }
-    return min(u1 - u0, max_per);
+    __syncthreads();
+    const int n = min(u1 - u0, max_per);
+    for (int e = tid; e < n; e += nthr) {
+        int32_t p = c.table[(int64_t)b * c.mbp + blk[e]];
+        if (p < 0 || p >= c.num_phys) {
+            set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
+            p = 0;
+            hm[e] = 0u;
+        }
+        phys[e] = p;
+    }
+    __syncthreads();
+    return n;
 }
 
 // Query-side constants, computed by nthr threads (tid in [0, nthr)); the caller
@@ -134,96 +153,92 @@ __device__ void query_phi(const CacheView& c, int b, int h, const float* qs, con
     for (int e = tid; e < G * d; e += nthr) aw[e] = expf(qs[e] + mrow[e % d] - cg[e / d]);
 }
 
-// Slice [r0, r1) of the global readout: nsl[g][j] = sum_i aw[g][i] S[i][j], dsl[g] = sum_i aw[g][i] z[i].
-__device__ void state_slice(const CacheView& c, int b, int h, int r0, int r1, const float* aw,
-                            float* nsl, float* dsl, int tid, int nthr) {
-    const int G = c.group, d = c.d;
-    const float* Sg = c.S + ((int64_t)b * c.hkv + h) * d * d;
-    const float* zg = c.z + ((int64_t)b * c.hkv + h) * d;
-    for (int j = tid; j < d; j += nthr) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int i = r0; i < r1; ++i) {
-            const float sv = Sg[(int64_t)i * d + j];
-#pragma unroll
-            for (int g = 0; g < 4; ++g)
-                if (g < G) acc[g] = fmaf(aw[g * d + i], sv, acc[g]);
-        }
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-            if (g < G) nsl[g * d + j] = acc[g];
-    }
-    const int warp = tid >> 5, lane = tid & 31;
-    if (warp < G) {
-        float s = 0.f;
-        for (int i = r0 + lane; i < r1; i += 32) s = fmaf(aw[warp * d + i], zg[i], s);
-        s = warp_sum(s);
-        if (lane == 0) dsl[warp] = s;
-    }
+// ------------------------------------------------------------------ group combine
+// Scratch floats the combine needs (16-byte aligned base).
+__host__ __device__ constexpr int combine_scratch_floats(int nsplit, int d) {
+    return 32 + 16 * nsplit + 4 * (d + 4) + 4 * nsplit + 8 * d;
 }
 
-// ------------------------------------------------------------------ group combine
-// Run by the last CTA of a (sequence, KV head) group. scr: >= 4*nsplit + 8*d + 32 floats.
+// Merges a (sequence, KV head) group's records with its global readout N, D.
+// Two rounds of loads only: first the record headers, the readout and the
+// selection counts, then every split's acc and N~ columns.
 template <typename T>
 __device__ void combine_group(const CacheView& c, const DecodeArgs& a, int b, int h, float* scr,
                               int tid, int nthr) {
     const int G = c.group, d = c.d, REC = rec_floats(d), ns = a.nsplit;
     const float* recs = a.part + ((int64_t)b * c.hkv + h) * ns * G * REC;   // [ns][G][REC]
-    float* sM = scr;            // [4]
-    float* sL = sM + 4;         // [4]
-    float* sD = sL + 4;         // [4]
-    float* sQ = sD + 4;         // [4] 1/rms of o_rla
-    float* fac = sQ + 4 + 16;   // [4][ns]
-    float* orl = fac + 4 * ns;  // [4][d]
-    float* osp = orl + 4 * d;   // [4][d]
+    const float* gr = a.gread + ((int64_t)b * c.hkv + h) * G * (d + 4);   // [G][d+4]
+    float* sM = scr;                                   // [4]
+    float* sL = sM + 4;                                // [4]
+    float* sD = sL + 4;                                // [4]  D - D~
+    float* sQ = sD + 4;                                // [4]  1/rms of o_rla
+    int* sN = reinterpret_cast<int*>(sQ + 4);          // [4]  kept-block counts
+    float4* hdr = reinterpret_cast<float4*>(scr + 32);  // [ns][G] record headers
+    float* grs = scr + 32 + 4 * ns * G;                // [G][d+4] readout N, D
+    float* fac = grs + G * (d + 4);                    // [4][ns]
+    float* orl = fac + 4 * ns;                         // [4][d]
+    float* osp = orl + 4 * d;                          // [4][d]
     const int warp = tid >> 5, lane = tid & 31;
     int32_t L = c.lens[b];
     L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + c.bs - 1) / c.bs;
+    // round 1
+    for (int e = tid; e < ns * G; e += nthr) hdr[e] = __ldcg(reinterpret_cast<const float4*>(recs + (int64_t)e * REC));
+    for (int e = tid; e < G * (d + 4); e += nthr) grs[e] = __ldcg(gr + e);
+    if (tid < G) sN[tid] = a.nsel[(int64_t)b * c.hq + h * G + tid];
+    __syncthreads();
     if (warp < G) {
         const int g = warp;
         float M = -SPLA_INF;
-        for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldcg(recs + ((int64_t)s * G + g) * REC));
+        for (int s = lane; s < ns; s += 32) M = fmaxf(M, hdr[s * G + g].x);
         M = warp_max(M);
-        float l = 0.f, dr = 0.f;
+        float l = 0.f, dt = 0.f;
         for (int s = lane; s < ns; s += 32) {
-            const float* r = recs + ((int64_t)s * G + g) * REC;
-            const float f = (M == -SPLA_INF) ? 0.f : ex2(__ldcg(r) - M);
+            const float4 r = hdr[s * G + g];
+            const float f = (M == -SPLA_INF) ? 0.f : ex2(r.x - M);
             fac[g * ns + s] = f;
-            l += __ldcg(r + 1) * f;
-            dr += __ldcg(r + 2);
+            l += r.y * f;
+            dt += r.z;
         }
         l = warp_sum(l);
-        dr = warp_sum(dr);
+        dt = warp_sum(dt);
         if (lane == 0) {
             sM[g] = M;
             sL[g] = l;
-            sD[g] = dr;
+            sD[g] = grs[g * (d + 4) + d] - dt;            // D - D~
         }
+    }
+    __syncthreads();
+    // round 2: sum the splits' acc (rescaled) and N~ fields, one float4 column per thread
+    const int d4 = d / 4;
+    for (int col = tid; col < G * 2 * d4; col += nthr) {
+        const int g = col / (2 * d4), part = (col / d4) & 1, j4 = col % d4;
+        const float* base = recs + (int64_t)g * REC + 4 + part * d + 4 * j4;
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int s = 0; s < ns; ++s) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(base + (int64_t)s * G * REC));
+            const float f = part ? 1.f : fac[g * ns + s];
+            t.x = fmaf(v.x, f, t.x);
+            t.y = fmaf(v.y, f, t.y);
+            t.z = fmaf(v.z, f, t.z);
+            t.w = fmaf(v.w, f, t.w);
+        }
+        float* dst = (part ? orl : osp) + g * d + 4 * j4;
+        dst[0] = t.x;
+        dst[1] = t.y;
+        dst[2] = t.z;
+        dst[3] = t.w;
     }
     __syncthreads();
     for (int e = tid; e < G * d; e += nthr) {
         const int g = e / d, j = e % d;
-        float o0 = 0.f, o1 = 0.f, R0 = 0.f, R1 = 0.f;
-        int s = 0;
-        for (; s + 1 < ns; s += 2) {
-            const float* r = recs + ((int64_t)s * G + g) * REC;
-            const float* r2 = r + (int64_t)G * REC;
-            o0 = fmaf(__ldcg(r + 4 + j), fac[g * ns + s], o0);
-            o1 = fmaf(__ldcg(r2 + 4 + j), fac[g * ns + s + 1], o1);
-            R0 += __ldcg(r + 4 + d + j);
-            R1 += __ldcg(r2 + 4 + d + j);
-        }
-        if (s < ns) {
-            const float* r = recs + ((int64_t)s * G + g) * REC;
-            o0 = fmaf(__ldcg(r + 4 + j), fac[g * ns + s], o0);
-            R0 += __ldcg(r + 4 + d + j);
-        }
         const float lsum = sL[g], Dr = sD[g];
-        const int hq = h * G + g;
-        const bool all_sel = a.nsel[(int64_t)b * c.hq + hq] >= nb;
+        const bool all_sel = sN[g] >= nb;
         const bool off = a.no_rla || all_sel || !(Dr > 0.f) || L == 0;
-        osp[e] = (lsum > 0.f) ? (o0 + o1) / lsum : 0.f;
-        orl[e] = off ? 0.f : (R0 + R1) / Dr;
+        osp[e] = (lsum > 0.f) ? osp[e] / lsum : 0.f;
+        const float R = grs[g * (d + 4) + j] - orl[e];             // N - N~
+        orl[e] = off ? 0.f : R / Dr;
     }
     __syncthreads();
     if (warp < G) {
@@ -244,22 +259,14 @@ __device__ void combine_group(const CacheView& c, const DecodeArgs& a, int b, in
     }
 }
 
-// Count this CTA in; the last one of the group combines (fence, then counter).
+// One CTA per (sequence, KV head) group merges the group's records: launched
+// after the decode kernel (programmatic dependent launch), it waits for it.
 template <typename T>
-__device__ void finish_group(const CacheView& c, const DecodeArgs& a, int b, int h, float* scr,
-                             int tid, int nthr, int* s_flag) {
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const int old = atomicAdd(&a.counters[(int64_t)b * c.hkv + h], 1);
-        *s_flag = (old == a.nsplit - 1);
-    }
-    __syncthreads();
-    if (*s_flag) {
-        __threadfence();
-        combine_group<T>(c, a, b, h, scr, tid, nthr);
-        if (tid == 0) a.counters[(int64_t)b * c.hkv + h] = 0;
-    }
+__global__ void __launch_bounds__(128) combine_kernel(CacheView c, const DecodeArgs a) {
+    extern __shared__ __align__(16) float smem_comb[];
+    pdl_wait();
+    const int b = blockIdx.x / c.hkv, h = blockIdx.x % c.hkv;
+    combine_group<T>(c, a, b, h, smem_comb, threadIdx.x, blockDim.x);
 }
 
 // ------------------------------------------------------------------ bf16 tensor-core kernel
@@ -275,7 +282,7 @@ struct MmaCfg {
 };
 
 template <int D, int UPB, int STAGES>
-__global__ void __launch_bounds__(MmaCfg<D, UPB, STAGES>::THREADS, 2)
+__global__ void __launch_bounds__(MmaCfg<D, UPB, STAGES>::THREADS, 3)
 decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const DecodeArgs a) {
     using Cfg = MmaCfg<D, UPB, STAGES>;
@@ -294,14 +301,14 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         (reinterpret_cast<uintptr_t>(hm + a.max_per) + 15) & ~uintptr_t(15));   // [4][D]
     float* aw = qs + G4 * D;                                // [4][D]
     float* ml = aw + G4 * D;                                // [D]
-    float* nsl = ml + D;                                    // [4][D]
-    float* dsl = nsl + G4 * D;                              // [4]
-    float* cg = dsl + G4;                                   // [4]
-    __shared__ int s_nblk, s_abort, s_flag;
+    float* cg = ml + D;                                     // [4]
+    __shared__ int s_n[2], s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv, split = blockIdx.x;
     const int G = c.group, nsplit = a.nsplit;
+    pdl_trigger();
+    pdl_wait();
     int32_t L = c.lens[b];
     if (L < 0 || L > c.mbp * c.bs) L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + BS - 1) / BS;
@@ -316,28 +323,18 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         fence_barrier_init();
         s_abort = 0;
     }
-    if (warp == NCW) {
-        const int n = (nb > 0) ? build_union_share(c, a.bits, a.nw, b, h, nb, split, nsplit,
-                                                   a.max_per, blk, phys, hm, a.status)
-                               : 0;
-        if (lane == 0) s_nblk = n;
-    } else if (nb > 0) {
-        query_load(c, a.q, 1, b, h, qs, ml, tid, NCW * 32);
-        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
-        query_max(c, b, h, qs, cg, tid);
-        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
-        query_phi(c, b, h, qs, cg, aw, tid, NCW * 32);
-    }
-    __syncthreads();
-    const int nblk = s_nblk;
+    // the union share first (all threads; the word counts borrow stage 0, no TMA yet)
+    const int nblk = (nb > 0) ? build_union_share(c, a.bits, a.nw, b, h, nb, split, nsplit,
+                                                  a.max_per, blk, phys, hm,
+                                                  reinterpret_cast<int*>(stages), s_n, a.status,
+                                                  tid, blockDim.x)
+                              : 0;
 
     if (nb == 0) {
         for (int e = tid; e < G * REC; e += blockDim.x) {
             const int g = e / REC, f = e % REC;
             a.part[(rec_base + g) * REC + f] = (f == 0) ? -SPLA_INF : 0.f;
         }
-        finish_group<__nv_bfloat16>(c, a, b, h, reinterpret_cast<float*>(stages), tid, blockDim.x,
-                                    &s_flag);
         return;
     }
 
@@ -351,6 +348,7 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     if (warp == NCW) {
         // ---------------- producer: TMA ring over 64-token units
         if (lane == 0) {
+            fence_proxy_async();   // stage 0 held the union word counts (generic writes)
             int u = 0;
             for (int it = 0; it < nblk && !s_abort; ++it) {
                 for (int half = 0; half < UPB; ++half) {
@@ -375,10 +373,13 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
             }
         }
     } else {
-        // ---------------- consumers
-        const int r0 = (int)((int64_t)split * D / nsplit);
-        const int r1 = (int)((int64_t)(split + 1) * D / nsplit);
-        state_slice(c, b, h, r0, r1, aw, nsl, dsl, tid, NCW * 32);
+        // ---------------- consumers: query constants while the first tiles land
+        query_load(c, a.q, 1, b, h, qs, ml, tid, NCW * 32);
+        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
+        query_max(c, b, h, qs, cg, tid);
+        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
+        query_phi(c, b, h, qs, cg, aw, tid, NCW * 32);
+        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
         // B fragments: column n = lane/4; rows k = 2*(lane%4) (+1, +8, +9) of each 16-dim step
         uint32_t qf[D / 16][2], wf[D / 16][2];
         {
@@ -435,15 +436,16 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
                         fence_proxy_async();
                         __syncwarp();
                     }
-                    float cl[4] = {0.f, 0.f, 0.f, 0.f}, cw1[4] = {0.f, 0.f, 0.f, 0.f},
-                          cw2[4] = {0.f, 0.f, 0.f, 0.f};
+                    // two logit accumulators (even/odd 16-dim steps) halve the MMA chain
+                    float cl[4] = {0.f, 0.f, 0.f, 0.f}, cl2[4] = {0.f, 0.f, 0.f, 0.f};
+                    float cw1[4] = {0.f, 0.f, 0.f, 0.f}, cw2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const int t = t0 + rr + ((qm & 1) << 3);
                         const int ch = ((kk & 3) << 1) + (qm >> 1);
                         uint32_t a0, a1, a2, a3;
                         ldsm_x4(kbase + (kk >> 2) * Cfg::BOX_BYTES + swz128(t, ch), a0, a1, a2, a3);
-                        mma_bf16(cl, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                        mma_bf16((kk & 1) ? cl2 : cl, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
                         const int kb = kk * 16 + 2 * (lane & 3);
                         const float2 mA = *reinterpret_cast<const float2*>(ml + kb);
                         const float2 mB = *reinterpret_cast<const float2*>(ml + kb + 8);
@@ -463,6 +465,8 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
                     }
                     // W = hi-part columns + lo-part columns (cols g and g+4)
                     float x[4], y[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) cl[r] += cl2[r];
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
                         x[r] = cw1[r] + cw2[r];
@@ -584,16 +588,14 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         }
         float* rec = a.part + (rec_base + g) * REC;
         rec[4 + j] = o;
-        rec[4 + D + j] = nsl[g * D + j] - nt;
+        rec[4 + D + j] = nt;
         if (j == 0) {
             rec[0] = M;
             rec[1] = l;
-            rec[2] = dsl[g] - dt;
+            rec[2] = dt;
             rec[3] = 0.f;
         }
     }
-    // scratch for the combine lies past the merge area
-    finish_group<__nv_bfloat16>(c, a, b, h, an + NCW * 4 * D, tid, blockDim.x, &s_flag);
 }
 
 // ------------------------------------------------------------------ fp32 SIMT kernel
@@ -610,19 +612,19 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const Dec
     float* qs = Ws + 4 * BS;                                // [4][d]
     float* aw = qs + 4 * d;                                 // [4][d]
     float* ml = aw + 4 * d;                                 // [d]
-    float* nsl = ml + d;                                    // [4][d]
-    float* dsl = nsl + 4 * d;                               // [4]
-    float* cg = dsl + 4;                                    // [4]
+    float* cg = ml + d;                                     // [4]
     float* fsc = cg + 4;                                    // [4] per-head rescale of this tile
     int32_t* blk = reinterpret_cast<int32_t*>(fsc + 4);
     int32_t* phys = blk + a.max_per;
     uint32_t* hm = reinterpret_cast<uint32_t*>(phys + a.max_per);
-    __shared__ int s_nblk, s_flag;
+    __shared__ int s_n[2];
     __shared__ float s_m[4], s_l[4], s_dt[4];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv, split = blockIdx.x;
     const int nsplit = a.nsplit;
+    pdl_trigger();
+    pdl_wait();
     int32_t L = c.lens[b];
     if (L < 0 || L > c.mbp * c.bs) L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + BS - 1) / BS;
@@ -633,14 +635,12 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const Dec
             const int g = e / REC, f = e % REC;
             a.part[(rec_base + g) * REC + f] = (f == 0) ? -SPLA_INF : 0.f;
         }
-        finish_group<T>(c, a, b, h, Ks, tid, blockDim.x, &s_flag);
         return;
     }
-    if (warp == 0) {
-        const int n = build_union_share(c, a.bits, a.nw, b, h, nb, split, nsplit, a.max_per, blk,
-                                        phys, hm, a.status);
-        if (lane == 0) s_nblk = n;
-    }
+    // union share (all threads; the word counts borrow the K tile)
+    const int nblk = build_union_share(c, a.bits, a.nw, b, h, nb, split, nsplit, a.max_per, blk,
+                                       phys, hm, reinterpret_cast<int*>(Ks), s_n, a.status, tid,
+                                       blockDim.x);
     query_load(c, a.q, sizeof(T) == 2, b, h, qs, ml, tid, blockDim.x);
     __syncthreads();
     query_max(c, b, h, qs, cg, tid);
@@ -648,9 +648,6 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const Dec
     query_phi(c, b, h, qs, cg, aw, tid, blockDim.x);
     if (tid < 4) { s_m[tid] = -SPLA_INF; s_l[tid] = 0.f; s_dt[tid] = 0.f; }
     __syncthreads();
-    const int r0 = (int)((int64_t)split * d / nsplit), r1 = (int)((int64_t)(split + 1) * d / nsplit);
-    state_slice(c, b, h, r0, r1, aw, nsl, dsl, tid, blockDim.x);
-    const int nblk = s_nblk;
     // accumulators: thread owns (g, j) pairs e = tid + 256*u
     constexpr int PU = 2;                                   // G*d <= 512
     float acc[PU] = {0.f, 0.f}, ntl[PU] = {0.f, 0.f};
@@ -736,17 +733,15 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const Dec
             const int g = e / d, j = e % d;
             float* rec = a.part + (rec_base + g) * REC;
             rec[4 + j] = acc[u];
-            rec[4 + d + j] = nsl[e] - ntl[u];
+            rec[4 + d + j] = ntl[u];
             if (j == 0) {
                 rec[0] = s_m[g];
                 rec[1] = s_l[g];
-                rec[2] = dsl[g] - s_dt[g];
+                rec[2] = s_dt[g];
                 rec[3] = 0.f;
             }
         }
     }
-    __syncthreads();
-    finish_group<T>(c, a, b, h, Ks, tid, blockDim.x, &s_flag);
 }
 
 // ------------------------------------------------------------------ host launchers
@@ -754,7 +749,7 @@ template <int D, int UPB, int STAGES>
 static size_t mma_smem_bytes(int max_per) {
     using Cfg = MmaCfg<D, UPB, STAGES>;
     return 1024 + (size_t)STAGES * Cfg::STAGE_BYTES + 2 * STAGES * sizeof(uint64_t) +
-           3 * (size_t)max_per * 4 + 16 + (size_t)(4 * D * 2 + D + 4 * D + 8) * 4 + 64;
+           3 * (size_t)max_per * 4 + 16 + (size_t)(4 * D * 2 + D + 4) * 4 + 64;
 }
 
 template <int D, int UPB, int STAGES>
@@ -765,38 +760,36 @@ static cudaError_t launch_mma_t(const CacheView& c, const CUtensorMap& tk, const
     cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D, UPB, STAGES>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    // all of the unified L1/shared array as shared memory: three CTAs per SM need it
+    e = cudaFuncSetAttribute(decode_mma_kernel<D, UPB, STAGES>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
     dim3 grid(a.nsplit, c.batch * c.hkv);
-    decode_mma_kernel<D, UPB, STAGES><<<grid, Cfg::THREADS, smem, s>>>(c, tk, tv, a);
-    return cudaGetLastError();
+    return launch_pdl(decode_mma_kernel<D, UPB, STAGES>, grid, dim3(Cfg::THREADS), smem, s, c, tk,
+                      tv, a);
 }
 
-// The merge area plus the combine scratch reuse the stage ring; they must fit
-// (nsplit is at most kMaxSplit, see the host layout).
+// The merge area reuses the stage ring; it must fit.
 constexpr int kMaxSplit = 512;
-static_assert(3 * MmaCfg<128, 1, 3>::STAGE_BYTES >=
-                  (2 * 4 * 4 * 128 + 48 + 32 + 4 * kMaxSplit + 8 * 128) * 4,
-              "stage ring too small for the merge and combine scratch");
-static_assert(4 * MmaCfg<64, 1, 4>::STAGE_BYTES >=
-                  (2 * 4 * 4 * 64 + 48 + 32 + 4 * kMaxSplit + 8 * 64) * 4,
-              "stage ring too small for the merge and combine scratch");
+static_assert(2 * MmaCfg<128, 1, 2>::STAGE_BYTES >= (2 * 4 * 4 * 128 + 64) * 4, "merge area");
+static_assert(4 * MmaCfg<64, 1, 4>::STAGE_BYTES >= (2 * 4 * 4 * 64 + 64) * 4, "merge area");
 
 size_t mma_smem_for(int d, int bs, int max_per) {
-    if (d == 128) return bs == 64 ? mma_smem_bytes<128, 1, 3>(max_per) : mma_smem_bytes<128, 2, 3>(max_per);
+    if (d == 128) return bs == 64 ? mma_smem_bytes<128, 1, 2>(max_per) : mma_smem_bytes<128, 2, 2>(max_per);
     return bs == 64 ? mma_smem_bytes<64, 1, 4>(max_per) : mma_smem_bytes<64, 2, 4>(max_per);
 }
 
 cudaError_t launch_decode_mma(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
                               const DecodeArgs& a, cudaStream_t s) {
-    if (c.d == 128 && c.bs == 64) return launch_mma_t<128, 1, 3>(c, tk, tv, a, s);
-    if (c.d == 128 && c.bs == 128) return launch_mma_t<128, 2, 3>(c, tk, tv, a, s);
+    if (c.d == 128 && c.bs == 64) return launch_mma_t<128, 1, 2>(c, tk, tv, a, s);
+    if (c.d == 128 && c.bs == 128) return launch_mma_t<128, 2, 2>(c, tk, tv, a, s);
     if (c.d == 64 && c.bs == 64) return launch_mma_t<64, 1, 4>(c, tk, tv, a, s);
     return launch_mma_t<64, 2, 4>(c, tk, tv, a, s);
 }
 
 size_t simt_smem_for(int d, int bs, int max_per) {
-    const size_t tiles = (size_t)(2 * bs * d + 8 * bs + 4 * d * 3 + d + 16) * 4;
-    const size_t comb = (size_t)(48 + 32 + 4 * kMaxSplit + 8 * d) * 4;   // combine scratch in Ks
-    return (tiles > comb ? tiles : comb) + 3 * (size_t)max_per * 4 + 64;
+    const size_t tiles = (size_t)(2 * bs * d + 8 * bs + 4 * d * 2 + d + 8) * 4;
+    return tiles + 3 * (size_t)max_per * 4 + 64;
 }
 
 cudaError_t launch_decode_simt(const CacheView& c, int dtype, const DecodeArgs& a, cudaStream_t s) {
@@ -807,14 +800,29 @@ cudaError_t launch_decode_simt(const CacheView& c, int dtype, const DecodeArgs& 
         e = cudaFuncSetAttribute(decode_simt_kernel<__nv_bfloat16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_simt_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(c, a);
+        return launch_pdl(decode_simt_kernel<__nv_bfloat16>, grid, dim3(256), smem, s, c, a);
     } else {
         e = cudaFuncSetAttribute(decode_simt_kernel<float>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_simt_kernel<float><<<grid, 256, smem, s>>>(c, a);
+        return launch_pdl(decode_simt_kernel<float>, grid, dim3(256), smem, s, c, a);
     }
-    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CacheView& c, int dtype, const DecodeArgs& a, cudaStream_t s) {
+    const size_t smem = (size_t)combine_scratch_floats(a.nsplit, c.d) * sizeof(float);
+    cudaError_t e;
+    if (dtype == SPLA_BF16) {
+        e = cudaFuncSetAttribute(combine_kernel<__nv_bfloat16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(c.batch * c.hkv), dim3(128), smem, s,
+                          c, a);
+    }
+    e = cudaFuncSetAttribute(combine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(combine_kernel<float>, dim3(c.batch * c.hkv), dim3(128), smem, s, c, a);
 }
 
 }  // namespace spla

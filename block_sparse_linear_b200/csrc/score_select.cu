@@ -4,34 +4,144 @@
 // exp(q.kbar)(1 + 1/2 q^T diag(sigma^2) q); the blocks with the largest
 // estimates are attended exactly).
 //
-// score_kernel  grid (chunks, batch*Hkv), 4 warps. Streams each block's
-//               statistics (1 KiB at d=128) once per KV head and scores it for
-//               all G query heads of the group. Lane l of a warp owns block
-//               jb + l: it walks the block's mean and variance in 16-byte
-//               loads and accumulates the G x 2 dot products in fp64 against
-//               {q', q'^2} broadcast from shared memory (no cross-lane work);
-//               the log-domain score is finished per lane.
+// score_kernel  grid (chunks + 1, batch*Hkv), 4 compute warps + 1 producer.
+//               Streams each block's statistics (1 KiB at d=128, stored in
+//               logical block order, so a CTA's range is contiguous) once per
+//               KV head through a 4-stage ring of 16 KiB bulk copies (TMA, no
+//               multicast), and scores every block for all G query heads of
+//               the group: lanes split the head dimension, form the 16 fp64
+//               partial dot products (2 blocks x 4 heads x 2 orders) and reduce
+//               them across lanes with a transposing butterfly that leaves
+//               value l in lanes l and l+16. The extra CTA of each group
+//               computes the global linear-attention readout N, D (it needs no
+//               selection).
 // select_kernel grid (batch*Hq), 512 threads. Exact top-k by key-space
 //               bucketing: 2048 linear buckets over the live key range, the
 //               bucket holding the k-th key is refined until few candidates
 //               remain, which are ranked pairwise (ties -> lower block index).
 //               Writes a per-head selection bitset (warp ballots over 32
-//               consecutive blocks), the sorted block list and its length, and
-//               clears the group's completion counter for the decode kernel.
+//               consecutive blocks), the sorted block list and its length.
 #include "common.cuh"
 
 namespace spla {
 
-constexpr int kScoreThreads = 128;     // 4 warps; a warp scores 32 blocks at once
+constexpr int kScoreBatch = 2;         // blocks a warp reduces together
+
+// 16 values per lane -> lanes l and l^16 end with the warp-wide sum of value
+// (l & 15) (fp64). At each level a lane keeps the half of its values whose index
+// has the lane's bit set (or clear) and adds the partner's copy of that half.
+__device__ __forceinline__ double transpose_reduce16(double (&v)[16]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int m = 8; m >= 1; m >>= 1) {
+        const bool up = lane & m;
+#pragma unroll
+        for (int i = 0; i < m; ++i) {
+            const double send = up ? v[i] : v[i + m];
+            const double keep = up ? v[i + m] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 16);
+}
+
+constexpr int kReadoutWarps = 4;       // warps of the score CTA that compute the readout
+
+// Global linear-attention readout of one (sequence, KV head) for its G query
+// heads (linear attention over all blocks, technical summary section 2.2):
+// N[g][j] = sum_i a_g,i S[i][j], D[g] = sum_i a_g,i z_i with
+// a_g,i = exp(q_g,i + m_i - c_g), c_g = max_i (q_g,i + m_i). Warps split the rows.
+template <int D, typename T>
+__device__ void global_readout(const CacheView& c, const T* __restrict__ q, int b, int h,
+                               float* __restrict__ gread, float* sm) {
+    const int G = c.group, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int nwarp = kReadoutWarps;   // the calling threads: warps 0..nwarp-1
+    float* aw = sm;                 // [4][D]
+    float* red = aw + 4 * D;        // [nwarp][4][D + 1]
+    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * D;
+    for (int e = threadIdx.x; e < 4 * D; e += nwarp * 32) {
+        const int g = e / D, i = e % D;
+        aw[e] = (g < G) ? to_f(q[((int64_t)b * c.hq + h * G + g) * D + i]) + mrow[i] : -SPLA_INF;
+    }
+    asm volatile("bar.sync 1, %0;" :: "r"(nwarp * 32));
+    if (warp < G) {
+        float mx = -SPLA_INF;
+        for (int i = lane; i < D; i += 32) mx = fmaxf(mx, aw[warp * D + i]);
+        mx = warp_max(mx);
+        __syncwarp();
+        for (int i = lane; i < D; i += 32) aw[warp * D + i] = expf(aw[warp * D + i] - mx);
+    }
+    asm volatile("bar.sync 1, %0;" :: "r"(nwarp * 32));
+    const float* Sg = c.S + ((int64_t)b * c.hkv + h) * D * D;
+    const float* zg = c.z + ((int64_t)b * c.hkv + h) * D;
+    constexpr int CPL = D / 32;     // columns per lane
+    float acc[4][CPL], dacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) acc[g][u] = 0.f;
+    const int rows = D / nwarp;
+#pragma unroll 4
+    for (int r = 0; r < rows; ++r) {
+        const int i = warp * rows + r;
+        float sv[CPL];
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) sv[u] = __ldg(Sg + (int64_t)i * D + lane + 32 * u);
+        const float zi = __ldg(zg + i);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            if (g < G) {
+                const float ag = aw[g * D + i];
+#pragma unroll
+                for (int u = 0; u < CPL; ++u) acc[g][u] = fmaf(ag, sv[u], acc[g][u]);
+                dacc[g] = fmaf(ag, zi, dacc[g]);
+            }
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) red[(warp * 4 + g) * (D + 1) + lane + 32 * u] = acc[g][u];
+        if (lane == 0) red[(warp * 4 + g) * (D + 1) + D] = dacc[g];
+    }
+    asm volatile("bar.sync 1, %0;" :: "r"(nwarp * 32));
+    float* out = gread + ((int64_t)b * c.hkv + h) * G * (D + 4);
+    for (int e = threadIdx.x; e < G * (D + 1); e += nwarp * 32) {
+        const int g = e / (D + 1), j = e % (D + 1);
+        float t = 0.f;
+        for (int w = 0; w < nwarp; ++w) t += red[(w * 4 + g) * (D + 1) + j];
+        out[g * (D + 4) + j] = t;
+    }
+}
+
+// Grid (chunks + 1, batch*Hkv): CTAs x < chunks score a contiguous range of
+// blocks, CTA x == chunks computes the group's global readout. A group's
+// statistics are contiguous (logical block order), so the producer warp moves a
+// whole stage of kScoreStageBlocks blocks with one bulk copy; the four compute
+// warps take kScoreStageBlocks/4 blocks each, two at a time.
+constexpr int kScoreStageBlocks = 16;
+constexpr int kScoreStages = 4;
+constexpr int kScoreWarps = 4;
 
 template <int D, typename T>
-__global__ void __launch_bounds__(kScoreThreads) score_kernel(CacheView c, const T* __restrict__ q,
-                                                              double scale, int first_order,
-                                                              float* __restrict__ scores,
-                                                              int chunk, int32_t* status) {
-    __shared__ double2 qsm[4][D];                  // {q', q'^2} per head and dimension
+__global__ void __launch_bounds__((kScoreWarps + 1) * 32, 3)
+score_kernel(CacheView c, const T* __restrict__ q, double scale, int first_order,
+             float* __restrict__ scores, int chunk, int nchunks, float* __restrict__ gread,
+             int32_t* status) {
+    constexpr int DPL = D / 32;                    // dimensions per lane: 2 or 4
+    constexpr int REC = 2 * D;                     // floats of one block's statistics
+    constexpr int STAGE = kScoreStageBlocks * REC; // floats per ring stage
+    extern __shared__ __align__(128) float smem_score[];
+    __shared__ uint64_t full[kScoreStages], empty[kScoreStages];
     const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    pdl_trigger();
+    pdl_wait();
+    if ((int)blockIdx.x == nchunks) {
+        static_assert(kReadoutWarps <= kScoreWarps, "readout warps");
+        if (threadIdx.x < kReadoutWarps * 32) global_readout<D, T>(c, q, b, h, gread, smem_score);
+        return;
+    }
     int32_t L = c.lens[b];
     if (L < 0 || L > c.mbp * c.bs) {
         if (blockIdx.x == 0 && threadIdx.x == 0 && h == 0) set_status(status, SPLA_DEV_CAPACITY);
@@ -41,59 +151,104 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(CacheView c, const
     const int j0 = blockIdx.x * chunk;
     if (j0 >= nb) return;
     const int j1 = min(nb, j0 + chunk);
+    const int nstage = (j1 - j0 + kScoreStageBlocks - 1) / kScoreStageBlocks;
     const int G = c.group;
-    for (int e = threadIdx.x; e < 4 * D; e += blockDim.x) {
-        const int g = e / D, i = e % D;
-        double v = 0.0;
-        if (g < G) v = (double)to_f(q[((int64_t)b * c.hq + h * G + g) * D + i]) * scale;
-        qsm[g][i] = make_double2(v, v * v);
+    const float* src = c.stats + (((int64_t)b * c.hkv + h) * c.mbp + j0) * REC;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kScoreStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kScoreWarps);
+        }
+        fence_barrier_init();
     }
     __syncthreads();
-    const int nwarps = blockDim.x >> 5;
-    for (int jb = j0 + warp * 32; jb < j1; jb += 32 * nwarps) {
-        const int j = jb + lane;
-        bool ok = false;
-        const float* st = c.stats;
-        if (j < j1) {
-            const int32_t phys = c.table[(int64_t)b * c.mbp + j];
-            ok = phys >= 0 && phys < c.num_phys;
-            if (ok) st = c.stats + ((int64_t)phys * c.hkv + h) * 2 * D;
-            else set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
-        }
-        double s1[4] = {0.0, 0.0, 0.0, 0.0}, s2[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 4
-        for (int i0 = 0; i0 < D; i0 += 4) {
-            float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f), v4 = m4;
-            if (ok) {
-                m4 = __ldg(reinterpret_cast<const float4*>(st + i0));
-                v4 = __ldg(reinterpret_cast<const float4*>(st + D + i0));
+
+    if (warp == kScoreWarps) {
+        // ---------------- producer
+        if (lane == 0) {
+            for (int t = 0; t < nstage; ++t) {
+                const int st = t % kScoreStages;
+                if (t >= kScoreStages && !mbar_wait_bounded(&empty[st], ((t / kScoreStages) - 1) & 1)) {
+                    set_status(status, SPLA_DEV_TIMEOUT);
+                    break;
+                }
+                const int nblk = min(kScoreStageBlocks, j1 - j0 - t * kScoreStageBlocks);
+                const uint32_t bytes = (uint32_t)nblk * REC * 4;
+                mbar_arrive_expect_tx(&full[st], bytes);
+                bulk_load(smem_score + st * STAGE, src + (int64_t)t * STAGE, bytes, &full[st]);
             }
-            const float mu[4] = {m4.x, m4.y, m4.z, m4.w}, va[4] = {v4.x, v4.y, v4.z, v4.w};
+        }
+        return;
+    }
+
+    // ---------------- compute warps
+    double qd[4][DPL], q2[4][DPL];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const double dm = (double)mu[u], dv = (double)va[u];
+    for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int u = 0; u < DPL; ++u) {
+            double v = 0.0;
+            if (g < G) v = (double)to_f(q[((int64_t)b * c.hq + h * G + g) * D + lane * DPL + u]) * scale;
+            qd[g][u] = v;
+            q2[g][u] = v * v;
+        }
+    constexpr int PER_WARP = kScoreStageBlocks / kScoreWarps;   // blocks of a stage per warp
+    const double log_bs = log((double)c.bs);
+    for (int t = 0; t < nstage; ++t) {
+        const int st = t % kScoreStages;
+        if (!mbar_wait_bounded(&full[st], (t / kScoreStages) & 1)) {
+            set_status(status, SPLA_DEV_TIMEOUT);
+            break;
+        }
+        const float* sb = smem_score + st * STAGE;
+#pragma unroll
+        for (int bb = 0; bb < PER_WARP; bb += kScoreBatch) {
+            double v[8 * kScoreBatch];
+#pragma unroll
+            for (int k = 0; k < kScoreBatch; ++k) {
+                const float* rec = sb + (warp * PER_WARP + bb + k) * REC;
+                float mu[DPL], va[DPL];
+                if constexpr (DPL == 4) {
+                    const float4 m4 = *reinterpret_cast<const float4*>(rec + lane * 4);
+                    const float4 v4 = *reinterpret_cast<const float4*>(rec + D + lane * 4);
+                    mu[0] = m4.x; mu[1] = m4.y; mu[2] = m4.z; mu[3] = m4.w;
+                    va[0] = v4.x; va[1] = v4.y; va[2] = v4.z; va[3] = v4.w;
+                } else {
+                    const float2 m2 = *reinterpret_cast<const float2*>(rec + lane * 2);
+                    const float2 v2 = *reinterpret_cast<const float2*>(rec + D + lane * 2);
+                    mu[0] = m2.x; mu[1] = m2.y;
+                    va[0] = v2.x; va[1] = v2.y;
+                }
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
-                    if (g < G) {
-                        const double2 qq = qsm[g][i0 + u];
-                        s1[g] = fma(qq.x, dm, s1[g]);
-                        s2[g] = fma(qq.y, dv, s2[g]);
-                    }
-                }
-            }
-        }
-        if (j < j1) {
-            const int nj = min(c.bs, L - j * c.bs);
-            const double ln = log((double)nj);
+                    double s1 = 0.0, s2 = 0.0;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                if (g < G) {
-                    double sc = ln + s1[g];
-                    if (!first_order) sc += log1p(0.5 * s2[g]);
-                    scores[((int64_t)b * c.hq + h * G + g) * c.mbp + j] = ok ? (float)sc : -SPLA_INF;
+                    for (int u = 0; u < DPL; ++u) {
+                        s1 = fma(qd[g][u], (double)mu[u], s1);
+                        s2 = fma(q2[g][u], (double)va[u], s2);
+                    }
+                    v[8 * k + 2 * g] = s1;
+                    v[8 * k + 2 * g + 1] = s2;
                 }
             }
+            const double tot = transpose_reduce16(v);
+            const double t2 = __shfl_down_sync(0xffffffffu, tot, 1);
+            const int k = (lane >> 3) & 1, g = (lane >> 1) & 3;
+            const int j = j0 + t * kScoreStageBlocks + warp * PER_WARP + bb + k;
+            if (lane < 16 && !(lane & 1) && g < G && j < j1) {
+                const int nj = min(c.bs, L - j * c.bs);
+                // log n_j: a constant except for a sequence's last block
+                double sc = ((nj == c.bs) ? log_bs : log((double)nj)) + tot;
+                if (!first_order) {
+                    // log1p in fp32 where it is accurate to ~6e-8 absolute (argument <= 1)
+                    const double x = 0.5 * t2;
+                    sc += (x <= 1.0) ? (double)log1pf((float)x) : log1p(x);
+                }
+                scores[((int64_t)b * c.hq + h * G + g) * c.mbp + j] = (float)sc;
+            }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
     }
 }
 
@@ -134,7 +289,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
                                                              int n_local, const float* scores,
                                                              uint32_t* bits, int nw,
                                                              int32_t* nsel, int32_t* sel_idx,
-                                                             int kcap, int32_t* counters) {
+                                                             int kcap) {
     extern __shared__ __align__(16) unsigned char smem_sel[];
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem_sel);        // [mbp padded]
     __shared__ int hist[kBins];
@@ -148,7 +303,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
 
     const int b = blockIdx.x / c.hq, hq = blockIdx.x % c.hq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0 && hq % c.group == 0) counters[(int64_t)b * c.hkv + hq / c.group] = 0;
+    pdl_trigger();
+    pdl_wait();
     int32_t L = c.lens[b];
     L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + c.bs - 1) / c.bs;
@@ -338,42 +494,45 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
     if (tid == 0) nsel[(int64_t)b * c.hq + hq] = total;
 }
 
-// ------------------------------------------------------------------ host launchers
+template <int D, typename T>
+static cudaError_t launch_score_t(const CacheView& c, const void* q, double scale, int first_order,
+                                  float* scores, int chunk, float* gread, int32_t* status,
+                                  cudaStream_t s) {
+    const int nchunks = (c.mbp + chunk - 1) / chunk;
+    const size_t ring = (size_t)kScoreStages * kScoreStageBlocks * 2 * D * sizeof(float);
+    const size_t rd = (size_t)(4 * D + kScoreWarps * 4 * (D + 1)) * sizeof(float);
+    const size_t smem = ring > rd ? ring : rd;
+    cudaError_t e = cudaFuncSetAttribute(score_kernel<D, T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(score_kernel<D, T>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    dim3 grid(nchunks + 1, c.batch * c.hkv);
+    return launch_pdl(score_kernel<D, T>, grid, dim3((kScoreWarps + 1) * 32), smem, s, c,
+                      (const T*)q, scale, first_order, scores, chunk, nchunks, gread, status);
+}
+
 cudaError_t launch_score(const CacheView& c, int dtype, const void* q, double scale,
-                         int first_order, float* scores, int chunk, int32_t* status,
-                         cudaStream_t s) {
-    dim3 grid((c.mbp + chunk - 1) / chunk, c.batch * c.hkv);
-    if (dtype == SPLA_BF16) {
-        if (c.d == 128)
-            score_kernel<128, __nv_bfloat16><<<grid, kScoreThreads, 0, s>>>(c, (const __nv_bfloat16*)q, scale,
-                                                                 first_order, scores, chunk, status);
-        else
-            score_kernel<64, __nv_bfloat16><<<grid, kScoreThreads, 0, s>>>(c, (const __nv_bfloat16*)q, scale,
-                                                                first_order, scores, chunk, status);
-    } else {
-        if (c.d == 128)
-            score_kernel<128, float><<<grid, kScoreThreads, 0, s>>>(c, (const float*)q, scale, first_order,
-                                                         scores, chunk, status);
-        else
-            score_kernel<64, float><<<grid, kScoreThreads, 0, s>>>(c, (const float*)q, scale, first_order,
-                                                        scores, chunk, status);
-    }
-    return cudaGetLastError();
+                         int first_order, float* scores, int chunk, float* gread,
+                         int32_t* status, cudaStream_t s) {
+    if (dtype == SPLA_BF16)
+        return c.d == 128 ? launch_score_t<128, __nv_bfloat16>(c, q, scale, first_order, scores, chunk, gread, status, s)
+                          : launch_score_t<64, __nv_bfloat16>(c, q, scale, first_order, scores, chunk, gread, status, s);
+    return c.d == 128 ? launch_score_t<128, float>(c, q, scale, first_order, scores, chunk, gread, status, s)
+                      : launch_score_t<64, float>(c, q, scale, first_order, scores, chunk, gread, status, s);
 }
 
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
                           const float* scores, uint32_t* bits, int nw, int32_t* nsel,
-                          int32_t* sel_idx, int kcap, int32_t* counters, cudaStream_t s) {
+                          int32_t* sel_idx, int kcap, cudaStream_t s) {
     const size_t smem = (size_t)((c.mbp + 31) / 32) * 32 * sizeof(uint32_t);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(select_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    select_kernel<<<c.batch * c.hq, kSelThreads, smem, s>>>(c, top_k, n_sink, n_local, scores,
-                                                            bits, nw, nsel, sel_idx, kcap,
-                                                            counters);
-    return cudaGetLastError();
+    return launch_pdl(select_kernel, dim3(c.batch * c.hq), dim3(kSelThreads), smem, s, c, top_k,
+                      n_sink, n_local, scores, bits, nw, nsel, sel_idx, kcap);
 }
 
 }  // namespace spla

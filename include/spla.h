@@ -90,8 +90,11 @@ typedef struct {
  * buffers are caller-allocated device memory; spla_cache_init prepares them.
  *   k_pool, v_pool : [num_phys_blocks][Hkv][B][d], params->dtype. Slots past a
  *                    sequence's length may hold anything.
- *   blk_stats      : [num_phys_blocks][Hkv][2][d] fp32: key mean, then key
- *                    population variance, of the block's stored tokens.
+ *   blk_stats      : [batch][Hkv][max_blocks_per_seq][2][d] fp32, indexed by
+ *                    LOGICAL block: key mean, then key population variance, of
+ *                    the block's stored tokens. Kept in logical order so that
+ *                    one sequence's statistics stream contiguously whatever the
+ *                    physical order of its KV blocks.
  *   S              : [batch][Hkv][d][d] fp32, sum_t exp(k_t - m) v_t^T
  *   z, m           : [batch][Hkv][d] fp32, sum_t exp(k_t - m) and the running
  *                    per-dimension max of k (the state's scaling).

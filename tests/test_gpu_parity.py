@@ -112,7 +112,7 @@ def test_append_state_matches_oracle():
         np.testing.assert_allclose(S[b, h], g.S, rtol=2e-5, atol=2e-5 * np.abs(g.S).max())
         n, mean, var = so.block_stats(g.K, w.block_size)
         for j in range(len(n)):
-            st = stats[table[b, j], h]
+            st = stats[b, h, j]
             np.testing.assert_allclose(st[0], mean[j], rtol=1e-6, atol=1e-7)
             np.testing.assert_allclose(st[1], var[j], rtol=1e-6, atol=1e-7)
 
