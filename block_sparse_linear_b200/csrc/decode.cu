@@ -17,10 +17,10 @@
 //     numerator and denominator (N~ = sum w v, D~ = sum w) with
 //     w_t = sum_i exp(q_i + m_i - c) exp(k_t,i - m_i);
 //   * writes one partial record per head: m, l, acc, N~, D~.
-// combine_kernel (one CTA per group, launched right behind) merges the group's
-// records: log-sum-exp merge of the softmax partials, o_rla = (N - N~)/(D - D~)
-// with the global readout N, D the scoring kernel computed from S, z;
-// RMSNorm; out = o_sparse + gamma * RMSNorm(o_rla).
+// combine_kernel (one CTA per query head, launched right behind) merges the
+// head's records: log-sum-exp merge of the softmax partials,
+// o_rla = (N - N~)/(D - D~) with the global readout N, D the scoring kernel
+// computed from S, z; RMSNorm; out = o_sparse + gamma * RMSNorm(o_rla).
 //
 // decode_mma_kernel (bf16 K/V): 4 consumer warps + 1 TMA producer warp, three
 // CTAs per SM (128 registers). The pipeline unit is a 64-token tile of one
@@ -153,120 +153,105 @@ __device__ void query_phi(const CacheView& c, int b, int h, const float* qs, con
     for (int e = tid; e < G * d; e += nthr) aw[e] = expf(qs[e] + mrow[e % d] - cg[e / d]);
 }
 
-// ------------------------------------------------------------------ group combine
-// Scratch floats the combine needs (16-byte aligned base).
-__host__ __device__ constexpr int combine_scratch_floats(int nsplit, int d) {
-    return 32 + 16 * nsplit + 4 * (d + 4) + 4 * nsplit + 8 * d;
-}
+// ------------------------------------------------------------------ combine
+// One CTA per (sequence, query head), thread j owns output column j. Every
+// thread issues its loads (the splits' acc[j] and N~[j], up to 32 splits at a
+// time, the readout N[j]) before any of them is needed; the record headers go
+// through shared memory. Launched right behind the decode kernel
+// (programmatic dependent launch), it waits for it.
+constexpr int kCombChunk = 32;
 
-// Merges a (sequence, KV head) group's records with its global readout N, D.
-// Two rounds of loads only: first the record headers, the readout and the
-// selection counts, then every split's acc and N~ columns.
-template <typename T>
-__device__ void combine_group(const CacheView& c, const DecodeArgs& a, int b, int h, float* scr,
-                              int tid, int nthr) {
-    const int G = c.group, d = c.d, REC = rec_floats(d), ns = a.nsplit;
-    const float* recs = a.part + ((int64_t)b * c.hkv + h) * ns * G * REC;   // [ns][G][REC]
-    const float* gr = a.gread + ((int64_t)b * c.hkv + h) * G * (d + 4);   // [G][d+4]
-    float* sM = scr;                                   // [4]
-    float* sL = sM + 4;                                // [4]
-    float* sD = sL + 4;                                // [4]  D - D~
-    float* sQ = sD + 4;                                // [4]  1/rms of o_rla
-    int* sN = reinterpret_cast<int*>(sQ + 4);          // [4]  kept-block counts
-    float4* hdr = reinterpret_cast<float4*>(scr + 32);  // [ns][G] record headers
-    float* grs = scr + 32 + 4 * ns * G;                // [G][d+4] readout N, D
-    float* fac = grs + G * (d + 4);                    // [4][ns]
-    float* orl = fac + 4 * ns;                         // [4][d]
-    float* osp = orl + 4 * d;                          // [4][d]
-    const int warp = tid >> 5, lane = tid & 31;
-    int32_t L = c.lens[b];
-    L = max(0, min(L, c.mbp * c.bs));
-    const int nb = (L + c.bs - 1) / c.bs;
-    // round 1
-    for (int e = tid; e < ns * G; e += nthr) hdr[e] = __ldcg(reinterpret_cast<const float4*>(recs + (int64_t)e * REC));
-    for (int e = tid; e < G * (d + 4); e += nthr) grs[e] = __ldcg(gr + e);
-    if (tid < G) sN[tid] = a.nsel[(int64_t)b * c.hq + h * G + tid];
-    __syncthreads();
-    if (warp < G) {
-        const int g = warp;
-        float M = -SPLA_INF;
-        for (int s = lane; s < ns; s += 32) M = fmaxf(M, hdr[s * G + g].x);
-        M = warp_max(M);
-        float l = 0.f, dt = 0.f;
-        for (int s = lane; s < ns; s += 32) {
-            const float4 r = hdr[s * G + g];
-            const float f = (M == -SPLA_INF) ? 0.f : ex2(r.x - M);
-            fac[g * ns + s] = f;
-            l += r.y * f;
-            dt += r.z;
-        }
-        l = warp_sum(l);
-        dt = warp_sum(dt);
-        if (lane == 0) {
-            sM[g] = M;
-            sL[g] = l;
-            sD[g] = grs[g * (d + 4) + d] - dt;            // D - D~
-        }
-    }
-    __syncthreads();
-    // round 2: sum the splits' acc (rescaled) and N~ fields, one float4 column per thread
-    const int d4 = d / 4;
-    for (int col = tid; col < G * 2 * d4; col += nthr) {
-        const int g = col / (2 * d4), part = (col / d4) & 1, j4 = col % d4;
-        const float* base = recs + (int64_t)g * REC + 4 + part * d + 4 * j4;
-        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int s = 0; s < ns; ++s) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(base + (int64_t)s * G * REC));
-            const float f = part ? 1.f : fac[g * ns + s];
-            t.x = fmaf(v.x, f, t.x);
-            t.y = fmaf(v.y, f, t.y);
-            t.z = fmaf(v.z, f, t.z);
-            t.w = fmaf(v.w, f, t.w);
-        }
-        float* dst = (part ? orl : osp) + g * d + 4 * j4;
-        dst[0] = t.x;
-        dst[1] = t.y;
-        dst[2] = t.z;
-        dst[3] = t.w;
-    }
-    __syncthreads();
-    for (int e = tid; e < G * d; e += nthr) {
-        const int g = e / d, j = e % d;
-        const float lsum = sL[g], Dr = sD[g];
-        const bool all_sel = sN[g] >= nb;
-        const bool off = a.no_rla || all_sel || !(Dr > 0.f) || L == 0;
-        osp[e] = (lsum > 0.f) ? osp[e] / lsum : 0.f;
-        const float R = grs[g * (d + 4) + j] - orl[e];             // N - N~
-        orl[e] = off ? 0.f : R / Dr;
-    }
-    __syncthreads();
-    if (warp < G) {
-        float sq = 0.f;
-        for (int j = lane; j < d; j += 32) sq = fmaf(orl[warp * d + j], orl[warp * d + j], sq);
-        sq = warp_sum(sq);
-        if (lane == 0) sQ[warp] = rsqrtf(sq / d + a.eps);
-    }
-    __syncthreads();
-    for (int e = tid; e < G * d; e += nthr) {
-        const int g = e / d, j = e % d;
-        const int hq = h * G + g;
-        const int64_t oi = ((int64_t)b * c.hq + hq) * d + j;
-        const float gm = a.gamma ? a.gamma[(int64_t)hq * d + j] : 1.f;
-        static_cast<T*>(a.out)[oi] = from_f<T>(osp[e] + gm * orl[e] * sQ[g]);
-        if (a.o_sp) a.o_sp[oi] = osp[e];
-        if (a.o_rl) a.o_rl[oi] = orl[e];
-    }
-}
-
-// One CTA per (sequence, KV head) group merges the group's records: launched
-// after the decode kernel (programmatic dependent launch), it waits for it.
 template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(CacheView c, const DecodeArgs a) {
     extern __shared__ __align__(16) float smem_comb[];
+    const int d = c.d, G = c.group, REC = rec_floats(d), ns = a.nsplit;
+    const int b = blockIdx.x / c.hq, hq = blockIdx.x % c.hq;
+    const int h = hq / G, g = hq % G;
+    const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
+    float* hdr = smem_comb;                 // [ns][4]: m, l, D~
+    float* fac = hdr + 4 * ns;              // [ns]
+    __shared__ float s_M, s_l, s_dt, s_D, s_red[4];
     pdl_wait();
-    const int b = blockIdx.x / c.hkv, h = blockIdx.x % c.hkv;
-    combine_group<T>(c, a, b, h, smem_comb, threadIdx.x, blockDim.x);
+    int32_t L = c.lens[b];
+    L = max(0, min(L, c.mbp * c.bs));
+    const int nb = (L + c.bs - 1) / c.bs;
+    const float* recs = a.part + (((int64_t)b * c.hkv + h) * ns * G + g) * REC;   // split s at s*G*REC
+    const float* gr = a.gread + (((int64_t)b * c.hkv + h) * G + g) * (d + 4);
+    for (int s = j; s < ns; s += blockDim.x)
+        reinterpret_cast<float4*>(hdr)[s] = __ldcg(reinterpret_cast<const float4*>(recs + (int64_t)s * G * REC));
+    const float Nj = __ldcg(gr + j);
+    if (j == 0) s_D = __ldcg(gr + d);
+    const int nsel = a.nsel[(int64_t)b * c.hq + hq];
+    // first chunk of columns in flight while the headers are reduced
+    float acc_v[kCombChunk], ntl_v[kCombChunk];
+#pragma unroll
+    for (int s = 0; s < kCombChunk; ++s) {
+        acc_v[s] = 0.f;
+        ntl_v[s] = 0.f;
+        if (s < ns) {
+            const float* r = recs + (int64_t)s * G * REC;
+            acc_v[s] = __ldcg(r + 4 + j);
+            ntl_v[s] = __ldcg(r + 4 + d + j);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        float M = -SPLA_INF;
+        for (int s = lane; s < ns; s += 32) M = fmaxf(M, hdr[4 * s]);
+        M = warp_max(M);
+        float l = 0.f, dt = 0.f;
+        for (int s = lane; s < ns; s += 32) {
+            const float f = (M == -SPLA_INF) ? 0.f : ex2(hdr[4 * s] - M);
+            fac[s] = f;
+            l += hdr[4 * s + 1] * f;
+            dt += hdr[4 * s + 2];
+        }
+        l = warp_sum(l);
+        dt = warp_sum(dt);
+        if (lane == 0) { s_M = M; s_l = l; s_dt = dt; }
+    }
+    __syncthreads();
+    float o = 0.f, nt = 0.f;
+#pragma unroll
+    for (int s = 0; s < kCombChunk; ++s)
+        if (s < ns) {
+            o = fmaf(acc_v[s], fac[s], o);
+            nt += ntl_v[s];
+        }
+    for (int s0 = kCombChunk; s0 < ns; s0 += kCombChunk) {
+#pragma unroll
+        for (int u = 0; u < kCombChunk; ++u) {
+            acc_v[u] = 0.f;
+            ntl_v[u] = 0.f;
+            if (s0 + u < ns) {
+                const float* r = recs + (int64_t)(s0 + u) * G * REC;
+                acc_v[u] = __ldcg(r + 4 + j);
+                ntl_v[u] = __ldcg(r + 4 + d + j);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kCombChunk; ++u)
+            if (s0 + u < ns) {
+                o = fmaf(acc_v[u], fac[s0 + u], o);
+                nt += ntl_v[u];
+            }
+    }
+    const float lsum = s_l, Dr = s_D - s_dt;
+    const bool off = a.no_rla || nsel >= nb || !(Dr > 0.f) || L == 0;
+    const float osp = (lsum > 0.f) ? o / lsum : 0.f;
+    const float orl = off ? 0.f : (Nj - nt) / Dr;
+    // RMS of o_rla over the head dimension
+    float sq = warp_sum(orl * orl);
+    if (lane == 0) s_red[warp] = sq;
+    __syncthreads();
+    sq = 0.f;
+    for (int w = 0; w < (d + 31) / 32; ++w) sq += s_red[w];
+    const float inv = rsqrtf(sq / d + a.eps);
+    const int64_t oi = ((int64_t)b * c.hq + hq) * d + j;
+    const float gm = a.gamma ? a.gamma[(int64_t)hq * d + j] : 1.f;
+    static_cast<T*>(a.out)[oi] = from_f<T>(osp + gm * orl * inv);
+    if (a.o_sp) a.o_sp[oi] = osp;
+    if (a.o_rl) a.o_rl[oi] = orl;
 }
 
 // ------------------------------------------------------------------ bf16 tensor-core kernel
@@ -810,19 +795,11 @@ cudaError_t launch_decode_simt(const CacheView& c, int dtype, const DecodeArgs& 
 }
 
 cudaError_t launch_combine(const CacheView& c, int dtype, const DecodeArgs& a, cudaStream_t s) {
-    const size_t smem = (size_t)combine_scratch_floats(a.nsplit, c.d) * sizeof(float);
-    cudaError_t e;
-    if (dtype == SPLA_BF16) {
-        e = cudaFuncSetAttribute(combine_kernel<__nv_bfloat16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(c.batch * c.hkv), dim3(128), smem, s,
-                          c, a);
-    }
-    e = cudaFuncSetAttribute(combine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(combine_kernel<float>, dim3(c.batch * c.hkv), dim3(128), smem, s, c, a);
+    const size_t smem = (size_t)5 * a.nsplit * sizeof(float);
+    const dim3 grid(c.batch * c.hq), block(c.d);
+    if (dtype == SPLA_BF16)
+        return launch_pdl(combine_kernel<__nv_bfloat16>, grid, block, smem, s, c, a);
+    return launch_pdl(combine_kernel<float>, grid, block, smem, s, c, a);
 }
 
 }  // namespace spla
