@@ -11,10 +11,11 @@ import torch
 
 from . import _lib
 from ._lib import (SPLA_BF16, SPLA_F32, SPLA_FLAG_FIRST_ORDER, SPLA_FLAG_NO_RLA, SplaError,
-                   spla_append_kv, spla_cache_init, spla_decode, spla_decode_workspace_size)
+                   spla_append_kv, spla_cache_init, spla_decode, spla_decode_static_workspace,
+                   spla_decode_workspace_size)
 
 __all__ = ["SplaConfig", "SplaDecodeCache", "SplaError", "spla_append_kv", "spla_cache_init",
-           "spla_decode", "spla_decode_workspace_size"]
+           "spla_decode", "spla_decode_static_workspace", "spla_decode_workspace_size"]
 
 
 @dataclass
@@ -112,6 +113,21 @@ class SplaDecodeCache:
         spla_decode(self.params, self.c, q.data_ptr(), ptr(gamma), out.data_ptr(), ptr(sel_idx),
                     ptr(o_sparse), ptr(o_rla), self.workspace.data_ptr(), self.ws_bytes,
                     self.dev_status.data_ptr(), self._stream(stream))
+        return out
+
+    def decode_static_workspace(self, q: torch.Tensor, gamma: torch.Tensor = None,
+                                out: torch.Tensor = None, sel_idx: torch.Tensor = None,
+                                o_sparse: torch.Tensor = None, o_rla: torch.Tensor = None,
+                                stream=None) -> torch.Tensor:
+        """decode() through spla_decode_static_workspace: the library's built-in scratch
+        instead of this object's workspace, for callers that cannot allocate per call."""
+        assert q.is_contiguous() and q.dtype == self.cfg.torch_dtype
+        if out is None:
+            out = torch.empty_like(q)
+        ptr = lambda t: 0 if t is None else t.data_ptr()
+        spla_decode_static_workspace(self.params, self.c, q.data_ptr(), ptr(gamma), out.data_ptr(),
+                                     ptr(sel_idx), ptr(o_sparse), ptr(o_rla),
+                                     self.dev_status.data_ptr(), self._stream(stream))
         return out
 
     def new_outputs(self, debug: bool = True):

@@ -29,9 +29,11 @@ SPLA_BF16 = 1
 SPLA_FLAG_NO_RLA = 0x1
 SPLA_FLAG_FIRST_ORDER = 0x2
 SPLA_MAX_BLOCKS_PER_SEQ = 32768
+SPLA_STATIC_WORKSPACE_BYTES = 16 << 20
 
 EXPORTS = ("spla_cache_init", "spla_append_kv", "spla_decode_workspace_size", "spla_decode",
-           "spla_profile_events", "spla_status_string", "spla_last_cuda_error", "spla_version")
+           "spla_decode_static_workspace", "spla_profile_events", "spla_status_string",
+           "spla_last_cuda_error", "spla_version")
 
 
 class spla_params(ctypes.Structure):
@@ -78,9 +80,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.spla_append_kv.argtypes = [P, C, vp, vp, vp, i32, vp, vp]
     lib.spla_decode_workspace_size.argtypes = [P, i32, i32, ctypes.POINTER(sz)]
     lib.spla_decode.argtypes = [P, C, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    lib.spla_decode_static_workspace.argtypes = [P, C, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.spla_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     for f in ("spla_cache_init", "spla_append_kv", "spla_decode_workspace_size", "spla_decode",
-              "spla_profile_events"):
+              "spla_decode_static_workspace", "spla_profile_events"):
         getattr(lib, f).restype = ctypes.c_int
     lib.spla_status_string.argtypes = [ctypes.c_int]
     lib.spla_status_string.restype = ctypes.c_char_p
@@ -120,6 +123,15 @@ def spla_decode(params, cache, q, rms_gamma, out, sel_idx, o_sparse_dbg, o_rla_d
     _check("spla_decode", load().spla_decode(ctypes.byref(params), ctypes.byref(cache), q,
                                              rms_gamma, out, sel_idx, o_sparse_dbg, o_rla_dbg,
                                              workspace, workspace_bytes, dev_status, stream))
+
+
+def spla_decode_static_workspace(params, cache, q, rms_gamma, out, sel_idx, o_sparse_dbg,
+                                 o_rla_dbg, dev_status, stream=0):
+    """spla_decode with the library's own scratch, for callers that cannot allocate."""
+    _check("spla_decode_static_workspace",
+           load().spla_decode_static_workspace(ctypes.byref(params), ctypes.byref(cache), q,
+                                               rms_gamma, out, sel_idx, o_sparse_dbg, o_rla_dbg,
+                                               dev_status, stream))
 
 
 def spla_profile_events(events):

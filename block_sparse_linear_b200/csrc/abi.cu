@@ -39,6 +39,8 @@ static void prof_mark(int i, cudaStream_t s) {
     if (g_prof_on) cudaEventRecord(g_prof[i], s);
 }
 
+void set_last_cuda_error(int32_t e) { g_last_cuda_error = e; }
+
 static spla_status cuda_fail(cudaError_t e) {
     g_last_cuda_error = (int32_t)e;
     return SPLA_ERR_CUDA;

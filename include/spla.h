@@ -172,6 +172,40 @@ SPLA_API spla_status spla_decode(const spla_params* params, const spla_cache* ca
                         int32_t* dev_status, void* stream);
 
 /*
+ * Bytes of the library-owned scratch that spla_decode_static_workspace uses
+ * on each device (one file-scope __device__ array, 256-byte aligned).
+ */
+#define SPLA_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/*
+ * spla_decode without a caller workspace: the method has no counterpart (the
+ * pages do not speak of memory management); this is a convenience of the
+ * library. It serves callers that cannot allocate device memory where they
+ * decode: a plain C host program with no device allocator of its own, or a
+ * serving engine whose KV-cache pool took all free HBM at start-up. It
+ * allocates nothing; the scratch is a SPLA_STATIC_WORKSPACE_BYTES array built
+ * into the library, one per device.
+ *   Arguments, results and dev_status are those of spla_decode; the work is
+ *   enqueued on `stream`, which must belong to the current device.
+ *   Size limit: a shape whose spla_decode_workspace_size exceeds
+ *   SPLA_STATIC_WORKSPACE_BYTES returns SPLA_ERR_CAPACITY on the host, before
+ *   any CUDA call, and enqueues nothing.
+ *   First call per device: it looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current, and keeps it; make that
+ *   first call before any stream capture on the device. A failed lookup
+ *   returns SPLA_ERR_CUDA.
+ *   Sharing: every call on a device uses the same array. Nothing in it needs
+ *   to start at zero (each kernel writes its scratch before the next one reads
+ *   it), so it is never cleared. Calls whose kernels overlap on the GPU (on
+ *   streams with no ordering between them) race on it.
+ */
+SPLA_API spla_status spla_decode_static_workspace(const spla_params* params,
+                                         const spla_cache* cache, const void* q,
+                                         const float* rms_gamma, void* out, int32_t* sel_idx,
+                                         float* o_sparse_dbg, float* o_rla_dbg,
+                                         int32_t* dev_status, void* stream);
+
+/*
  * Measurement hook (no part of the method). With n == 5, every later
  * spla_decode call made from this host thread records events[0..4]
  * (cudaEvent_t handles) on its stream: before the scoring kernel, after it,

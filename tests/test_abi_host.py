@@ -120,3 +120,21 @@ def test_python_binding_raises_on_error_codes():
     with pytest.raises(_lib.SplaError) as e:
         _lib.spla_decode_workspace_size(_params(head_dim=100), 1, 1)
     assert e.value.status == _lib.SPLA_ERR_UNSUPPORTED
+
+
+def test_static_workspace_entry_rejects_oversize_shapes_on_the_host(lib):
+    """spla_decode_static_workspace checks its fixed scratch size before any CUDA call."""
+    B = ctypes.byref
+    p = _params()
+    c = _cache(batch=64)
+    assert _lib.spla_decode_workspace_size(p, 64, 2064) > _lib.SPLA_STATIC_WORKSPACE_BYTES
+    assert lib.spla_decode_static_workspace(B(p), B(c), FAKE, None, FAKE, None, None, None, None,
+                                            None) == _lib.SPLA_ERR_CAPACITY
+    assert lib.spla_decode_static_workspace(B(p), None, FAKE, None, FAKE, None, None, None, None,
+                                            None) == _lib.SPLA_ERR_INVALID_ARG
+    bad = _params(head_dim=96)
+    assert lib.spla_decode_static_workspace(B(bad), B(_cache()), FAKE, None, FAKE, None, None,
+                                            None, None, None) == _lib.SPLA_ERR_UNSUPPORTED
+    with pytest.raises(_lib.SplaError) as e:
+        _lib.spla_decode_static_workspace(p, c, FAKE, 0, FAKE, 0, 0, 0, 0)
+    assert e.value.status == _lib.SPLA_ERR_CAPACITY
