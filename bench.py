@@ -145,12 +145,65 @@ def step_bytes(w, sel: np.ndarray, lens: np.ndarray) -> dict:
     return {"kv": kv, "stats": stats, "state": state, "total": kv + stats + state}
 
 
+# Kernel of each profiled phase, and the source file that defines it.
+KERNELS = {"score": ("score_kernel", "score_select.cu"),
+           "select": ("select_kernel", "score_select.cu"),
+           "decode": ("decode_mma_kernel", "decode.cu"),
+           "combine": ("combine_kernel", "decode.cu")}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+
+
+def source_digest(fname: str) -> str:
+    import hashlib
+    path = os.path.join(ROOT, "block_sparse_linear_b200", "csrc", fname)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(workload: str, context: int, phase: str):
+    """DRAM bytes (read + write) per launch of a phase's kernel, from an ncu capture
+    recorded in profiles/dram_traffic.txt; None unless that capture was taken on this
+    workload and on the kernel's current source."""
+    kname, fname = KERNELS[phase]
+    try:
+        digest = source_digest(fname)
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) != 6 or line.startswith("#"):
+                    continue
+                wl, ctx, kn, fn, dg, nbytes = parts
+                if (wl, int(ctx), kn, fn, dg) == (workload, context, kname, fname, digest):
+                    return int(float(nbytes))
+    except (OSError, ValueError):
+        return None
+    return None
+
+
 def workload_of(args):
     from workloads import gen
     if args.context > 0:
         w = gen.get(args.workload)
         return gen.scaled(args.workload, (args.context,) * w.batch, name=w.name)
     return gen.get(args.workload)
+
+
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(vals, dev):
+    """Element-wise max over all ranks of a list of floats (one all-reduce; the
+    identity without an initialised process group). Every rank must call it."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_value(world: int, units_per_step: int, steps: int, t_ms: float) -> float:
+    """Whole-job throughput: every rank processes its own batch of units each step."""
+    return world * units_per_step * steps / (t_ms / 1e3)
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -240,18 +293,12 @@ def run_ours(args):
     if not args.no_e2e:
         e2e = e2e_pass(w, cache, steps, W + 2 * K, K, gamma, flush, dev, stream, ones)
 
-    # ---- reduce over ranks
-    t_max = t_total
-    if world > 1:
-        tt = torch.tensor([t_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
-        if e2e is not None:
-            te = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-            e2e["ms"] = float(te.item())
+    # ---- max over ranks (the same single collective on every rank)
+    t_max, e2e_ms = max_over_ranks([t_total, e2e["ms"] if e2e is not None else 0.0], dev)
+    if e2e is not None:
+        e2e["ms"] = e2e_ms
     units_per_step = w.batch * w.num_q_heads
-    value = world * units_per_step * K / (t_max / 1e3)
+    value = job_value(world, units_per_step, K, t_max)
 
     if rank == 0:
         hbm, peak_kind = peaks()
@@ -259,8 +306,10 @@ def run_ours(args):
         sco = kt[:, 0]
         share = kt.sum(axis=0) / kt.sum()
         dom = int(np.argmax(share))
-        dec_bytes = np.mean([b["kv"] + b["state"] for b in byB])
-        sco_bytes = np.mean([b["stats"] for b in byB])
+        # the scoring kernel reads the statistics and the S, z, m state (global readout);
+        # the decode kernel reads the union of kept K/V
+        dec_bytes = np.mean([b["kv"] for b in byB])
+        sco_bytes = np.mean([b["stats"] + b["state"] for b in byB])
         dom_bytes = dec_bytes if dom == 2 else sco_bytes
         dom_ms = float(np.mean(kt[:, dom]))
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9
@@ -279,7 +328,9 @@ def run_ours(args):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": {"bound": "hbm", "kernel": kernel_names[dom],
                          "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(achieved / hbm, 4), "traffic": None,
+                         "frac": round(achieved / hbm, 4),
+                         "traffic": measured_traffic(w.name, int(w.context_lens[0]),
+                                                     kernel_names[dom]),
                          "peak_kind": f"{peak_kind} hbm_gbs",
                          "bytes_per_launch": int(dom_bytes), "ms_per_launch": round(dom_ms, 5)},
             "step_hbm": {"bytes_per_step": int(np.mean([b["total"] for b in by])),
@@ -291,11 +342,12 @@ def run_ours(args):
             "kernels_ms": {n: round(float(np.mean(kt[:, j])), 5) for j, n in enumerate(kernel_names)},
             "kernel_share": {n: round(float(share[j]), 4) for j, n in enumerate(kernel_names)},
             "clocks": clk.summary(),
-            "gpu_launches": 6 * K,
+            # per step: 3 append kernels + score, select, decode, combine
+            "gpu_launches": 7 * K,
             "dev_status": status,
         }
         if e2e is not None:
-            res["e2e"] = {"value": round(world * units_per_step * K / (e2e["ms"] / 1e3), 1),
+            res["e2e"] = {"value": round(job_value(world, units_per_step, K, e2e["ms"]), 1),
                           "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
                           "d2h_bytes_per_step": e2e["d2h"]}
         if not args.no_cpu_baseline:
@@ -385,8 +437,9 @@ def run_reference(args):
         return
     from workloads import gen
     w = workload_of(args)
-    oracle_sample(w, 0.0, steps=args.warmup)                  # warm-up (untimed)
-    v, units, secs, desc, n = oracle_sample(w, 0.0, steps=args.steps)
+    if args.warmup > 0:
+        oracle_sample(w, 0.0, steps=args.warmup)              # warm-up (untimed)
+    v, units, secs, desc, n = oracle_sample(w, 0.0, steps=max(1, args.steps))
     res = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT,
            "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(secs / n * 1e3, 3), "higher_is_better": True,
