@@ -11,9 +11,10 @@ namespace spla {
 cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s);
 cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, const void* v_new,
                           const int32_t* n_new, int32_t max_new, int32_t* status, cudaStream_t s);
-cudaError_t launch_score(const CacheView& c, int dtype, const void* q, double scale,
-                         int first_order, float* scores, int chunk, float* gread,
+cudaError_t launch_score(const CacheView& c, const CUtensorMap& tstats, int dtype, const void* q,
+                         double scale, int first_order, float* scores, float* gread,
                          int32_t* status, cudaStream_t s);
+int score_readout_parts(int d);
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
                           const float* scores, uint32_t* bits, int nw, int32_t* nsel,
                           int32_t* sel_idx, int kcap, cudaStream_t s);
@@ -107,11 +108,7 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     ns = std::max(1, std::min(ns, std::min(kMaxSplit, std::max(1, umax / 2))));
     L.nsplit = ns;
     L.max_per = (umax + ns - 1) / ns + 1;
-    // scoring chunk: 256 blocks per CTA; smaller while that leaves fewer than two
-    // CTAs per SM
-    int chunk = 256;
-    while (chunk > 32 && (int64_t)groups * ((mbp + chunk - 1) / chunk) < 2 * kTargetCtas) chunk >>= 1;
-    L.score_chunk = chunk;
+    L.readout_parts = score_readout_parts(p->head_dim);
     size_t off = 0;
     L.off_scores = off;
     off = align256(off + (size_t)batch * p->num_q_heads * mbp * sizeof(float));
@@ -122,7 +119,7 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     L.off_part = off;
     off = align256(off + (size_t)groups * ns * G * L.rec * sizeof(float));
     L.off_gread = off;
-    off = align256(off + (size_t)groups * G * (p->head_dim + 4) * sizeof(float));
+    off = align256(off + (size_t)groups * L.readout_parts * G * (p->head_dim + 4) * sizeof(float));
     L.total = off;
     return L;
 }
@@ -154,6 +151,21 @@ static bool make_pool_map(CUtensorMap* m, const void* pool, const CacheView& c) 
     cuuint32_t estr[2] = {1u, 1u};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 2-D view of the block statistics as [batch*Hkv*mbp rows][2d fp32 cols]; box = 32 rows x 32
+// cols (the mean or the variance of 32 dimensions of 32 blocks, 4 KiB), 128B swizzle.
+static bool make_stats_map(CUtensorMap* m, const CacheView& c) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(2 * c.d), (cuuint64_t)c.batch * c.hkv * c.mbp};
+    cuuint64_t strides[1] = {(cuuint64_t)(2 * c.d) * 4};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, c.stats, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -259,8 +271,10 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
 
     prof_mark(0, s);
     float* gread = reinterpret_cast<float*>(ws + L.off_gread);
-    cudaError_t e = launch_score(v, params->dtype, q, scale, first_order, scores, L.score_chunk,
-                                 gread, dev_status, s);
+    CUtensorMap tstats;
+    if (!make_stats_map(&tstats, v)) return cuda_fail(cudaErrorInvalidValue);
+    cudaError_t e = launch_score(v, tstats, params->dtype, q, scale, first_order, scores, gread,
+                                 dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(1, s);
     e = launch_select(v, params->top_k, params->n_sink, params->n_local, scores, bits, L.nw, nsel,
@@ -282,6 +296,7 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     da.nsplit = L.nsplit;
     da.max_per = L.max_per;
     da.no_rla = no_rla;
+    da.nrd = L.readout_parts;
     da.sl2 = sl2;
     da.eps = eps;
     if (use_mma) {

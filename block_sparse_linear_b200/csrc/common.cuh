@@ -11,6 +11,9 @@
 #define SPLA_INF __int_as_float(0x7f800000)
 #define SPLA_LOG2E 1.4426950408889634f
 
+// SMs of a B200; grids of persistent kernels are sized from it.
+constexpr int kNumSms = 148;
+
 namespace spla {
 
 // ------------------------------------------------------------------ launch-time description
@@ -34,7 +37,7 @@ struct DecodeLayout {
     int32_t nw;              // 32-bit words of a per-head selection bitset
     int32_t kcap;            // top_k + n_sink + n_local
     int32_t rec;             // floats per partial record
-    int32_t score_chunk;     // blocks per scoring CTA
+    int32_t readout_parts;   // row ranges of S the global readout is split into
     int32_t max_per;         // union blocks one decode CTA may receive
     size_t off_scores, off_bits, off_nsel, off_part, off_gread, total;
 };
@@ -49,9 +52,9 @@ struct DecodeArgs {
     const uint32_t* bits;       // [batch][Hq][nw] selection bitsets
     const int32_t* nsel;        // [batch][Hq]
     float* part;                // [batch*Hkv][nsplit][G][rec]
-    const float* gread;         // [batch*Hkv][G][d+4]: global readout N (d), then D
+    const float* gread;         // [batch*Hkv][nrd][G][d+4]: readout parts, N (d) then D
     int32_t* status;
-    int nw, nsplit, max_per, no_rla;
+    int nw, nsplit, max_per, no_rla, nrd;
     float sl2, eps;
 };
 
@@ -163,6 +166,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];"
         :: "r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y) : "memory");
+}
+
+// Bring a kernel-parameter tensor map into the TMA unit's descriptor cache.
+__device__ __forceinline__ void prefetch_tmap(const void* tmap) {
+    asm volatile("prefetch.tensormap [%0];" :: "l"(tmap) : "memory");
 }
 
 // 1-D bulk copy global -> this CTA's shared memory (16-byte aligned, size a

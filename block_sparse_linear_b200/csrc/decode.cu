@@ -176,11 +176,15 @@ __global__ void __launch_bounds__(128) combine_kernel(CacheView c, const DecodeA
     L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + c.bs - 1) / c.bs;
     const float* recs = a.part + (((int64_t)b * c.hkv + h) * ns * G + g) * REC;   // split s at s*G*REC
-    const float* gr = a.gread + (((int64_t)b * c.hkv + h) * G + g) * (d + 4);
+    const float* gr = a.gread + (((int64_t)b * c.hkv + h) * a.nrd * G + g) * (d + 4);
     for (int s = j; s < ns; s += blockDim.x)
         reinterpret_cast<float4*>(hdr)[s] = __ldcg(reinterpret_cast<const float4*>(recs + (int64_t)s * G * REC));
-    const float Nj = __ldcg(gr + j);
-    if (j == 0) s_D = __ldcg(gr + d);
+    float Nj = 0.f, Dg = 0.f;
+    for (int p = 0; p < a.nrd; ++p) {              // the readout's row-range parts add
+        Nj += __ldcg(gr + (int64_t)p * G * (d + 4) + j);
+        if (j == 0) Dg += __ldcg(gr + (int64_t)p * G * (d + 4) + d);
+    }
+    if (j == 0) s_D = Dg;
     const int nsel = a.nsel[(int64_t)b * c.hq + hq];
     // first chunk of columns in flight while the headers are reduced
     float acc_v[kCombChunk], ntl_v[kCombChunk];
@@ -293,6 +297,10 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv, split = blockIdx.x;
     const int G = c.group, nsplit = a.nsplit;
     pdl_trigger();
+    if (tid == 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
     pdl_wait();
     int32_t L = c.lens[b];
     if (L < 0 || L > c.mbp * c.bs) L = max(0, min(L, c.mbp * c.bs));

@@ -4,17 +4,12 @@
 // exp(q.kbar)(1 + 1/2 q^T diag(sigma^2) q); the blocks with the largest
 // estimates are attended exactly).
 //
-// score_kernel  grid (chunks + 1, batch*Hkv), 4 compute warps + 1 producer.
-//               Streams each block's statistics (1 KiB at d=128, stored in
-//               logical block order, so a CTA's range is contiguous) once per
-//               KV head through a 4-stage ring of 16 KiB bulk copies (TMA, no
-//               multicast), and scores every block for all G query heads of
-//               the group: lanes split the head dimension, form the 16 fp64
-//               partial dot products (2 blocks x 4 heads x 2 orders) and reduce
-//               them across lanes with a transposing butterfly that leaves
-//               value l in lanes l and l+16. The extra CTA of each group
-//               computes the global linear-attention readout N, D (it needs no
-//               selection).
+// score_kernel  persistent grid (2 CTAs of 4 warps per SM), every warp its
+//               own TMA pipeline over equal 32 KiB items: 32-block tiles of
+//               the statistics (lane l scores block l of the tile for all G
+//               heads with fp64 dot products, no lane reduction) and row
+//               ranges of the global state S for the linear-attention readout
+//               N, D that the combine step subtracts from.
 // select_kernel grid (batch*Hq), 512 threads. Exact top-k by key-space
 //               bucketing: 2048 linear buckets over the live key range, the
 //               bucket holding the k-th key is refined until few candidates
@@ -25,230 +20,379 @@
 
 namespace spla {
 
-constexpr int kScoreBatch = 2;         // blocks a warp reduces together
+// ------------------------------------------------------------------ scoring
+// One launch works through a list of equal-sized items, taken by the warps of a
+// persistent grid (warp w of NW takes items w, w + NW, ...):
+//   items [0, groups*RP)       global readout of one (sequence, KV head) group,
+//                              part p of RP row ranges of S (RP = 2 at d = 128);
+//   items groups*RP + gi*ntile + t
+//                              scores of blocks 32t .. 32t+31 of group gi.
+// Each warp is its own pipeline: lane 0 keeps kScoreRing stages of 8 KiB in
+// flight on per-warp mbarriers, the whole warp consumes them in order.
+//
+// Score tile: the statistics are a 2-D fp32 tensor [groups*mbp rows][2d] (mean,
+// then variance, logical block order); one stage is two 32 x 32 boxes (mean and
+// variance of 32 dimensions of 32 blocks) with 128-byte swizzle. The dot
+// products run on the fp64 tensor cores (mma m8n8k4 f64): A = 8 blocks x 4
+// dimensions of statistics, B = 4 dimensions x 8 columns, the columns being
+// q'_g (g < 4) and q'_g^2 (g >= 4), q' = q * softmax_scale. B stays in
+// registers for the whole group (D/4 fp64 per lane); mean tiles accumulate
+// into one C, variance tiles into another, and the useful halves (mean x q',
+// variance x q'^2) are paired across lanes at the end. Rows of an A fragment
+// are blocks r/2 + 4(r%2) of an 8-block group, which keeps every quarter
+// warp's 16-byte reads on distinct bank groups under the swizzle.
+//
+// Readout part: N[g][j] += sum_i a_g,i S[i][j], D[g] += sum_i a_g,i z_i over
+// its rows i, with a_g,i = exp(q_g,i + m_i - c_g), c_g = max over all i of
+// q_g,i + m_i (the same in every part, so the parts add). S rows arrive by 1-D
+// bulk copies; lane l owns columns l*d/32 ...
+//
+// Nothing on the streaming path is read with ordinary loads: while the memory
+// system is saturated with bulk traffic those take microseconds to return. An
+// item's query rows (and m, z for a readout) arrive by bulk copy on a second
+// per-warp barrier, issued with the item's first stage; sequence lengths are
+// read into shared memory once at the start.
+constexpr int kScoreWarps = 4;          // warps per CTA
+constexpr int kScoreRing = 2;           // stages in flight per warp
+constexpr int kScoreStage = 8192;       // bytes per stage
+constexpr int kScoreCtasPerSm = 2;
+constexpr int kTile = 32;               // blocks per score item
+constexpr int kScoreNbSmem = 512;       // sequences whose block counts are cached in smem
 
-// 16 values per lane -> lanes l and l^16 end with the warp-wide sum of value
-// (l & 15) (fp64). At each level a lane keeps the half of its values whose index
-// has the lane's bit set (or clear) and adds the partner's copy of that half.
-__device__ __forceinline__ double transpose_reduce16(double (&v)[16]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int m = 8; m >= 1; m >>= 1) {
-        const bool up = lane & m;
-#pragma unroll
-        for (int i = 0; i < m; ++i) {
-            const double send = up ? v[i] : v[i + m];
-            const double keep = up ? v[i + m] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-        }
-    }
-    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 16);
+template <int D>
+struct ScoreShape {
+    static constexpr int kTileStages = D / 32;                              // 32 dims per stage
+    static constexpr int kReadoutParts = (D * D * 4) / (kTileStages * kScoreStage);
+    static constexpr int kRowsPerStage = kScoreStage / (D * 4);
+    static constexpr int kATab = D * 4 * 4;                                 // readout weights [D][4]
+    // per-item inputs by bulk copy: the group's G query rows (up to 2 KiB), then m and z (D floats each)
+    static constexpr int kQBytes = 2048;
+    static constexpr int kAux = kQBytes + 2 * D * 4;
+    static constexpr int kAuxPad = 1024 * ((kAux + 1023) / 1024);
+    // two input buffers: item k uses buffer k % 2, so the next item's copy never
+    // lands in rows the current item still reads
+    static constexpr int kWarpBytes = kScoreRing * kScoreStage + kATab + 2 * kAuxPad;
+    static constexpr int kSmem = kScoreWarps * kWarpBytes + 1024;           // + alignment
+    static_assert(kReadoutParts >= 1 && kReadoutParts * kTileStages * kRowsPerStage == D, "parts");
+    static_assert(kWarpBytes % 1024 == 0, "ring alignment for the 128B swizzle");
+};
+
+// D(8x8, f64) += A(8x4, row) * B(4x8, col); per lane a = A[lane/4][lane%4],
+// b = B[lane%4][lane/4], c = D[lane/4][2(lane%4) .. +1].
+__device__ __forceinline__ void dmma_884(double (&c)[2], double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+                 : "+d"(c[0]), "+d"(c[1]) : "d"(a), "d"(b));
 }
 
-constexpr int kReadoutWarps = 4;       // warps of the score CTA that compute the readout
+// log n for n = 0 .. 128 (entry 0 unused): the log n_j term of a partial block.
+__constant__ double c_log_n[129] = {0.0, 0.0, 0.6931471805599453, 1.0986122886681098, 1.3862943611198906, 1.6094379124341003, 1.791759469228055, 1.9459101490553132, 2.0794415416798357, 2.1972245773362196, 2.302585092994046, 2.3978952727983707, 2.4849066497880004, 2.5649493574615367, 2.6390573296152584, 2.70805020110221, 2.772588722239781, 2.833213344056216, 2.8903717578961645, 2.9444389791664403, 2.995732273553991, 3.044522437723423, 3.091042453358316, 3.1354942159291497, 3.1780538303479458, 3.2188758248682006, 3.258096538021482, 3.295836866004329, 3.332204510175204, 3.367295829986474, 3.4011973816621555, 3.4339872044851463, 3.4657359027997265, 3.4965075614664802, 3.5263605246161616, 3.5553480614894135, 3.58351893845611, 3.6109179126442243, 3.6375861597263857, 3.6635616461296463, 3.6888794541139363, 3.713572066704308, 3.7376696182833684, 3.7612001156935624, 3.784189633918261, 3.8066624897703196, 3.828641396489095, 3.8501476017100584, 3.871201010907891, 3.8918202981106265, 3.912023005428146, 3.9318256327243257, 3.9512437185814275, 3.970291913552122, 3.9889840465642745, 4.007333185232471, 4.02535169073515, 4.04305126783455, 4.060443010546419, 4.07753744390572, 4.0943445622221, 4.110873864173311, 4.127134385045092, 4.143134726391533, 4.1588830833596715, 4.174387269895637, 4.189654742026425, 4.204692619390966, 4.219507705176107, 4.23410650459726, 4.248495242049359, 4.2626798770413155, 4.276666119016055, 4.290459441148391, 4.30406509320417, 4.31748811353631, 4.330733340286331, 4.343805421853684, 4.356708826689592, 4.3694478524670215, 4.382026634673881, 4.394449154672439, 4.406719247264253, 4.418840607796598, 4.430816798843313, 4.442651256490317, 4.454347296253507, 4.465908118654584, 4.477336814478207, 4.48863636973214, 4.499809670330265, 4.51085950651685, 4.5217885770490405, 4.532599493153256, 4.543294782270004, 4.553876891600541, 4.564348191467836, 4.574710978503383, 4.584967478670572, 4.59511985013459, 4.605170185988092, 4.61512051684126, 4.624972813284271, 4.634728988229636, 4.6443908991413725, 4.653960350157523, 4.663439094112067, 4.672828834461906, 4.68213122712422, 4.6913478822291435, 4.700480365792417, 4.709530201312334, 4.718498871295094, 4.727387818712341, 4.736198448394496, 4.74493212836325, 4.7535901911063645, 4.762173934797756, 4.770684624465665, 4.77912349311153, 4.787491742782046, 4.795790545596741, 4.804021044733257, 4.812184355372417, 4.820281565605037, 4.8283137373023015, 4.836281906951478, 4.844187086458591, 4.852030263919617};
 
-// Global linear-attention readout of one (sequence, KV head) for its G query
-// heads (linear attention over all blocks, technical summary section 2.2):
-// N[g][j] = sum_i a_g,i S[i][j], D[g] = sum_i a_g,i z_i with
-// a_g,i = exp(q_g,i + m_i - c_g), c_g = max_i (q_g,i + m_i). Warps split the rows.
-template <int D, typename T>
-__device__ void global_readout(const CacheView& c, const T* __restrict__ q, int b, int h,
-                               float* __restrict__ gread, float* sm) {
-    const int G = c.group, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int nwarp = kReadoutWarps;   // the calling threads: warps 0..nwarp-1
-    float* aw = sm;                 // [4][D]
-    float* red = aw + 4 * D;        // [nwarp][4][D + 1]
-    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * D;
-    for (int e = threadIdx.x; e < 4 * D; e += nwarp * 32) {
-        const int g = e / D, i = e % D;
-        aw[e] = (g < G) ? to_f(q[((int64_t)b * c.hq + h * G + g) * D + i]) + mrow[i] : -SPLA_INF;
+template <typename T> struct QVec;
+template <> struct QVec<__nv_bfloat16> {
+    // 4 consecutive bf16 values (8 bytes) as floats
+    static __device__ __forceinline__ void load4(const __nv_bfloat16* p, float (&v)[4]) {
+        const uint2 u = *reinterpret_cast<const uint2*>(p);
+        v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
     }
-    asm volatile("bar.sync 1, %0;" :: "r"(nwarp * 32));
-    if (warp < G) {
-        float mx = -SPLA_INF;
-        for (int i = lane; i < D; i += 32) mx = fmaxf(mx, aw[warp * D + i]);
-        mx = warp_max(mx);
-        __syncwarp();
-        for (int i = lane; i < D; i += 32) aw[warp * D + i] = expf(aw[warp * D + i] - mx);
+};
+template <> struct QVec<float> {
+    static __device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
+        const float4 u = *reinterpret_cast<const float4*>(p);
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
     }
-    asm volatile("bar.sync 1, %0;" :: "r"(nwarp * 32));
-    const float* Sg = c.S + ((int64_t)b * c.hkv + h) * D * D;
-    const float* zg = c.z + ((int64_t)b * c.hkv + h) * D;
-    constexpr int CPL = D / 32;     // columns per lane
-    float acc[4][CPL], dacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int g = 0; g < 4; ++g)
-#pragma unroll
-        for (int u = 0; u < CPL; ++u) acc[g][u] = 0.f;
-    const int rows = D / nwarp;
-#pragma unroll 4
-    for (int r = 0; r < rows; ++r) {
-        const int i = warp * rows + r;
-        float sv[CPL];
-#pragma unroll
-        for (int u = 0; u < CPL; ++u) sv[u] = __ldg(Sg + (int64_t)i * D + lane + 32 * u);
-        const float zi = __ldg(zg + i);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            if (g < G) {
-                const float ag = aw[g * D + i];
-#pragma unroll
-                for (int u = 0; u < CPL; ++u) acc[g][u] = fmaf(ag, sv[u], acc[g][u]);
-                dacc[g] = fmaf(ag, zi, dacc[g]);
-            }
-        }
-    }
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-#pragma unroll
-        for (int u = 0; u < CPL; ++u) red[(warp * 4 + g) * (D + 1) + lane + 32 * u] = acc[g][u];
-        if (lane == 0) red[(warp * 4 + g) * (D + 1) + D] = dacc[g];
-    }
-    asm volatile("bar.sync 1, %0;" :: "r"(nwarp * 32));
-    float* out = gread + ((int64_t)b * c.hkv + h) * G * (D + 4);
-    for (int e = threadIdx.x; e < G * (D + 1); e += nwarp * 32) {
-        const int g = e / (D + 1), j = e % (D + 1);
-        float t = 0.f;
-        for (int w = 0; w < nwarp; ++w) t += red[(w * 4 + g) * (D + 1) + j];
-        out[g * (D + 4) + j] = t;
-    }
-}
-
-// Grid (chunks + 1, batch*Hkv): CTAs x < chunks score a contiguous range of
-// blocks, CTA x == chunks computes the group's global readout. A group's
-// statistics are contiguous (logical block order), so the producer warp moves a
-// whole stage of kScoreStageBlocks blocks with one bulk copy; the four compute
-// warps take kScoreStageBlocks/4 blocks each, two at a time.
-constexpr int kScoreStageBlocks = 16;
-constexpr int kScoreStages = 4;
-constexpr int kScoreWarps = 4;
+};
 
 template <int D, typename T>
-__global__ void __launch_bounds__((kScoreWarps + 1) * 32, 3)
-score_kernel(CacheView c, const T* __restrict__ q, double scale, int first_order,
-             float* __restrict__ scores, int chunk, int nchunks, float* __restrict__ gread,
-             int32_t* status) {
-    constexpr int DPL = D / 32;                    // dimensions per lane: 2 or 4
-    constexpr int REC = 2 * D;                     // floats of one block's statistics
-    constexpr int STAGE = kScoreStageBlocks * REC; // floats per ring stage
-    extern __shared__ __align__(128) float smem_score[];
-    __shared__ uint64_t full[kScoreStages], empty[kScoreStages];
-    const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv;
+__global__ void __launch_bounds__(kScoreWarps * 32, kScoreCtasPerSm)
+score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* __restrict__ q,
+             double scale, double log_bs, int first_order, float* __restrict__ scores,
+             float* __restrict__ gread, int ntile, int32_t* status) {
+    using S = ScoreShape<D>;
+    constexpr int RP = S::kReadoutParts, TS = S::kTileStages, RPS = S::kRowsPerStage;
+    constexpr int CPL = D / 32;                    // readout columns per lane
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ uint64_t full[kScoreWarps][kScoreRing];
+    __shared__ uint64_t qfull[kScoreWarps][2];
+    __shared__ int s_nb[kScoreNbSmem], s_len[kScoreNbSmem];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    pdl_trigger();
-    pdl_wait();
-    if ((int)blockIdx.x == nchunks) {
-        static_assert(kReadoutWarps <= kScoreWarps, "readout warps");
-        if (threadIdx.x < kReadoutWarps * 32) global_readout<D, T>(c, q, b, h, gread, smem_score);
-        return;
-    }
-    int32_t L = c.lens[b];
-    if (L < 0 || L > c.mbp * c.bs) {
-        if (blockIdx.x == 0 && threadIdx.x == 0 && h == 0) set_status(status, SPLA_DEV_CAPACITY);
-        L = max(0, min(L, c.mbp * c.bs));
-    }
-    const int nb = (L + c.bs - 1) / c.bs;
-    const int j0 = blockIdx.x * chunk;
-    if (j0 >= nb) return;
-    const int j1 = min(nb, j0 + chunk);
-    const int nstage = (j1 - j0 + kScoreStageBlocks - 1) / kScoreStageBlocks;
+    unsigned char* base = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* ring = base + warp * S::kWarpBytes;
+    float* at = reinterpret_cast<float*>(ring + kScoreRing * kScoreStage);    // readout [D][4]
+    unsigned char* aux0 = ring + kScoreRing * kScoreStage + S::kATab;          // q rows, m, z (x2)
+    uint64_t* bar = full[warp];
+    uint64_t* qbar = qfull[warp];
     const int G = c.group;
-    const float* src = c.stats + (((int64_t)b * c.hkv + h) * c.mbp + j0) * REC;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kScoreStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kScoreWarps);
-        }
+    const int groups = c.batch * c.hkv;
+    const int nread = groups * RP;
+    const int nitems = nread + groups * ntile;
+    const int NW = gridDim.x * kScoreWarps;
+    const int wg = blockIdx.x * kScoreWarps + warp;
+
+    pdl_trigger();
+    if (threadIdx.x == 0) prefetch_tmap(&tstats);
+    if (lane == 0) {
+        for (int s = 0; s < kScoreRing; ++s) mbar_init(&bar[s], 1);
+        mbar_init(&qbar[0], 1);
+        mbar_init(&qbar[1], 1);
         fence_barrier_init();
     }
-    __syncthreads();
-
-    if (warp == kScoreWarps) {
-        // ---------------- producer
-        if (lane == 0) {
-            for (int t = 0; t < nstage; ++t) {
-                const int st = t % kScoreStages;
-                if (t >= kScoreStages && !mbar_wait_bounded(&empty[st], ((t / kScoreStages) - 1) & 1)) {
-                    set_status(status, SPLA_DEV_TIMEOUT);
-                    break;
-                }
-                const int nblk = min(kScoreStageBlocks, j1 - j0 - t * kScoreStageBlocks);
-                const uint32_t bytes = (uint32_t)nblk * REC * 4;
-                mbar_arrive_expect_tx(&full[st], bytes);
-                bulk_load(smem_score + st * STAGE, src + (int64_t)t * STAGE, bytes, &full[st]);
-            }
-        }
-        return;
+    pdl_wait();          // statistics, state and lengths come from the append kernels
+    for (int b = threadIdx.x; b < min(c.batch, kScoreNbSmem); b += blockDim.x) {
+        const int32_t L = c.lens[b];
+        if (blockIdx.x == 0 && (L < 0 || L > c.mbp * c.bs)) set_status(status, SPLA_DEV_CAPACITY);
+        s_len[b] = max(0, min(L, c.mbp * c.bs));
+        s_nb[b] = (s_len[b] + c.bs - 1) / c.bs;
     }
+    __syncthreads();
+    auto len_of = [&](int b) {
+        return b < kScoreNbSmem ? s_len[b] : max(0, min(c.lens[b], c.mbp * c.bs));
+    };
+    auto nb_of = [&](int b) {
+        if (b < kScoreNbSmem) return s_nb[b];
+        return (len_of(b) + c.bs - 1) / c.bs;
+    };
+    // next non-empty item at or after i in this warp's sequence
+    auto next_item = [&](int i) {
+        for (; i < nitems; i += NW) {
+            if (i < nread) return i;
+            const int r = i - nread, gi = r / ntile, t = r % ntile;
+            if (t * kTile < nb_of(gi / c.hkv)) return i;
+        }
+        return nitems;
+    };
 
-    // ---------------- compute warps
-    double qd[4][DPL], q2[4][DPL];
-#pragma unroll
-    for (int g = 0; g < 4; ++g)
-#pragma unroll
-        for (int u = 0; u < DPL; ++u) {
-            double v = 0.0;
-            if (g < G) v = (double)to_f(q[((int64_t)b * c.hq + h * G + g) * D + lane * DPL + u]) * scale;
-            qd[g][u] = v;
-            q2[g][u] = v * v;
+    // ---- producer state (lane 0): item, stage within it, stages issued
+    int pi = next_item(wg), ps = 0, fi = 0, pk = 0;     // pk: items issued
+    auto issue = [&]() {
+        if (pi >= nitems) return;
+        const int slot = fi % kScoreRing;
+        unsigned char* dst = ring + slot * kScoreStage;
+        if (ps == 0) {
+            // the item's query rows (and m, z for a readout) on the item barrier
+            const int gi = pi < nread ? pi / RP : (pi - nread) / ntile;
+            const int b = gi / c.hkv, h = gi % c.hkv;
+            const uint32_t qb = (uint32_t)(G * D * sizeof(T));
+            unsigned char* ax = aux0 + (pk & 1) * S::kAuxPad;
+            uint64_t* qb_bar = &qbar[pk & 1];
+            ++pk;
+            mbar_arrive_expect_tx(qb_bar, qb + (pi < nread ? 2u * D * 4u : 0u));
+            bulk_load(ax, q + ((int64_t)b * c.hq + h * G) * D, qb, qb_bar);
+            if (pi < nread) {
+                bulk_load(ax + S::kQBytes, c.m + (int64_t)gi * D, D * 4, qb_bar);
+                bulk_load(ax + S::kQBytes + D * 4, c.z + (int64_t)gi * D, D * 4, qb_bar);
+            }
         }
-    constexpr int PER_WARP = kScoreStageBlocks / kScoreWarps;   // blocks of a stage per warp
-    const double log_bs = log((double)c.bs);
-    for (int t = 0; t < nstage; ++t) {
-        const int st = t % kScoreStages;
-        if (!mbar_wait_bounded(&full[st], (t / kScoreStages) & 1)) {
-            set_status(status, SPLA_DEV_TIMEOUT);
-            break;
+        mbar_arrive_expect_tx(&bar[slot], kScoreStage);
+        if (pi < nread) {
+            const int gi = pi / RP, part = pi % RP;
+            const float* src = c.S + (int64_t)gi * D * D + ((int64_t)part * TS + ps) * RPS * D;
+            bulk_load(dst, src, kScoreStage, &bar[slot]);
+        } else {
+            const int r = pi - nread, gi = r / ntile, t = r % ntile;
+            const int y = gi * c.mbp + t * kTile;
+            tma_load_2d(dst, &tstats, &bar[slot], ps * 32, y);
+            tma_load_2d(dst + kScoreStage / 2, &tstats, &bar[slot], D + ps * 32, y);
         }
-        const float* sb = smem_score + st * STAGE;
+        ++fi;
+        if (++ps == TS) {
+            ps = 0;
+            pi = next_item(pi + NW);
+        }
+    };
+    if (lane == 0)
+        for (int s = 0; s < kScoreRing; ++s) issue();
+
+    int f = 0;                 // stages consumed
+    int nq = 0;                // items started: buffer nq % 2, its phase (nq / 2) % 2
+    // after a failed wait lane 0 waits (bounded) for every copy it has in flight
+    auto drain = [&](int q_from) {
+        set_status(status, SPLA_DEV_TIMEOUT);
+        for (int k = f; k < fi; ++k) mbar_wait_bounded(&bar[k % kScoreRing], (k / kScoreRing) & 1);
+        for (int k = q_from; k < pk; ++k) mbar_wait_bounded(&qbar[k & 1], (k >> 1) & 1);
+    };
+    // every lane agrees on the outcome of a wait
+    auto wait_stage = [&](int slot) -> bool {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar[slot], (f / kScoreRing) & 1));
+        if (!ok && lane == 0) drain(nq);
+        return ok;
+    };
+    const T* qs = nullptr;
+    const float* ms = nullptr;
+    const float* zs_ = nullptr;
+    auto wait_item = [&]() -> bool {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&qbar[nq & 1], (nq >> 1) & 1));
+        const unsigned char* ax = aux0 + (nq & 1) * S::kAuxPad;
+        qs = reinterpret_cast<const T*>(ax);
+        ms = reinterpret_cast<const float*>(ax + S::kQBytes);
+        zs_ = ms + D;
+        if (!ok && lane == 0) drain(nq);
+        ++nq;
+        return ok;
+    };
+    const int kq = lane & 3, rq = lane >> 2;
+
+    for (int i = next_item(wg); i < nitems; i = next_item(i + NW)) {
+        if (i < nread) {
+            // ---------------- global readout, rows of part `part`
+            const int gi = i / RP, part = i % RP;
+            float dsum[4];
+            if (!wait_item()) return;
+            __syncwarp();                  // the previous readout's reads of `at` are done
 #pragma unroll
-        for (int bb = 0; bb < PER_WARP; bb += kScoreBatch) {
-            double v[8 * kScoreBatch];
+            for (int g = 0; g < 4; ++g) {
+                dsum[g] = 0.f;
+                if (g < G) {
+                    float v[CPL], mx = -SPLA_INF;
 #pragma unroll
-            for (int k = 0; k < kScoreBatch; ++k) {
-                const float* rec = sb + (warp * PER_WARP + bb + k) * REC;
-                float mu[DPL], va[DPL];
-                if constexpr (DPL == 4) {
-                    const float4 m4 = *reinterpret_cast<const float4*>(rec + lane * 4);
-                    const float4 v4 = *reinterpret_cast<const float4*>(rec + D + lane * 4);
-                    mu[0] = m4.x; mu[1] = m4.y; mu[2] = m4.z; mu[3] = m4.w;
-                    va[0] = v4.x; va[1] = v4.y; va[2] = v4.z; va[3] = v4.w;
-                } else {
-                    const float2 m2 = *reinterpret_cast<const float2*>(rec + lane * 2);
-                    const float2 v2 = *reinterpret_cast<const float2*>(rec + D + lane * 2);
-                    mu[0] = m2.x; mu[1] = m2.y;
-                    va[0] = v2.x; va[1] = v2.y;
-                }
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    double s1 = 0.0, s2 = 0.0;
-#pragma unroll
-                    for (int u = 0; u < DPL; ++u) {
-                        s1 = fma(qd[g][u], (double)mu[u], s1);
-                        s2 = fma(q2[g][u], (double)va[u], s2);
+                    for (int u = 0; u < CPL; ++u) {
+                        const int r = lane + 32 * u;
+                        v[u] = to_f(qs[g * D + r]) + ms[r];
+                        mx = fmaxf(mx, v[u]);
                     }
-                    v[8 * k + 2 * g] = s1;
-                    v[8 * k + 2 * g + 1] = s2;
+                    mx = warp_max(mx);
+                    float zs = 0.f;
+#pragma unroll
+                    for (int u = 0; u < CPL; ++u) {
+                        const int r = lane + 32 * u;
+                        const float a = (mx == -SPLA_INF) ? 0.f : expf(v[u] - mx);
+                        at[r * 4 + g] = a;
+                        if (r / (D / RP) == part) zs = fmaf(a, zs_[r], zs);
+                    }
+                    dsum[g] = warp_sum(zs);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < CPL; ++u) at[(lane + 32 * u) * 4 + g] = 0.f;
                 }
             }
-            const double tot = transpose_reduce16(v);
-            const double t2 = __shfl_down_sync(0xffffffffu, tot, 1);
-            const int k = (lane >> 3) & 1, g = (lane >> 1) & 3;
-            const int j = j0 + t * kScoreStageBlocks + warp * PER_WARP + bb + k;
-            if (lane < 16 && !(lane & 1) && g < G && j < j1) {
+            __syncwarp();
+            float acc[4][CPL];
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+#pragma unroll
+                for (int u = 0; u < CPL; ++u) acc[g][u] = 0.f;
+#pragma unroll 1
+            for (int s = 0; s < TS; ++s, ++f) {
+                const int slot = f % kScoreRing;
+                if (!wait_stage(slot)) return;
+                const float* sm = reinterpret_cast<const float*>(ring + slot * kScoreStage);
+                const int row0 = (part * TS + s) * RPS;
+#pragma unroll 4
+                for (int r = 0; r < RPS; ++r) {
+                    const float4 a4 = *reinterpret_cast<const float4*>(at + (row0 + r) * 4);
+                    float sv[CPL];
+                    if constexpr (CPL == 4) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(sm + r * D + lane * 4);
+                        sv[0] = t4.x; sv[1] = t4.y; sv[2] = t4.z; sv[3] = t4.w;
+                    } else {
+                        const float2 t2 = *reinterpret_cast<const float2*>(sm + r * D + lane * 2);
+                        sv[0] = t2.x; sv[1] = t2.y;
+                    }
+                    const float ag[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+#pragma unroll
+                        for (int u = 0; u < CPL; ++u) acc[g][u] = fmaf(ag[g], sv[u], acc[g][u]);
+                }
+                __syncwarp();
+                if (lane == 0) issue();
+            }
+            float* out = gread + ((int64_t)gi * RP + part) * G * (D + 4);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                if (g < G) {
+#pragma unroll
+                    for (int u = 0; u < CPL; ++u) out[g * (D + 4) + lane * CPL + u] = acc[g][u];
+                    if (lane == 0) out[g * (D + 4) + D] = dsum[g];
+                }
+            }
+            continue;
+        }
+        // ---------------- score tile
+        const int r = i - nread, gi = r / ntile, t = r % ntile;
+        const int b = gi / c.hkv, h = gi % c.hkv;
+        if (!wait_item()) return;
+        double cm[4][2], cs[4][2];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) cm[m][0] = cm[m][1] = cs[m][0] = cs[m][1] = 0.0;
+        const int prow = (rq >> 1) + 4 * (rq & 1);          // block row of A row rq in a group of 8
+        const int head = rq & 3;
+        const bool sq = rq >= 4;
+        const T* qh = qs + head * D;
+        // one copy of the stage code (kept small: it runs cold at first, while the
+        // memory system is saturated)
+#pragma unroll 1
+        for (int s = 0; s < TS; ++s, ++f) {
+            // B[k][n] of k-slice (hf, u) is column n's query value at dimension
+            // 32s + 16hf + 4k + u: q'_n for n < 4, q'_{n-4}^2 for n >= 4, 0 past G.
+            double bq[8];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float v[4] = {0.f, 0.f, 0.f, 0.f};
+                if (head < G) QVec<T>::load4(qh + 32 * s + 16 * hf + 4 * kq, v);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const double x = (double)v[u] * scale;
+                    bq[hf * 4 + u] = sq ? x * x : x;
+                }
+            }
+            const int slot = f % kScoreRing;
+            if (!wait_stage(slot)) return;
+            const unsigned char* st = ring + slot * kScoreStage;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float mu[4][4], va[4][4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const uint32_t off = swz128(8 * m + prow, 4 * hf + kq);
+                    const float4 m4 = *reinterpret_cast<const float4*>(st + off);
+                    const float4 v4 = *reinterpret_cast<const float4*>(st + kScoreStage / 2 + off);
+                    mu[m][0] = m4.x; mu[m][1] = m4.y; mu[m][2] = m4.z; mu[m][3] = m4.w;
+                    va[m][0] = v4.x; va[m][1] = v4.y; va[m][2] = v4.z; va[m][3] = v4.w;
+                }
+                // eight independent accumulators per k-slice
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        dmma_884(cm[m], (double)mu[m][u], bq[hf * 4 + u]);
+                        dmma_884(cs[m], (double)va[m][u], bq[hf * 4 + u]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) issue();
+        }
+        // lanes kq < 2 hold mean x q' (columns 2kq, 2kq+1 = heads); their partners
+        // kq + 2 hold variance x q'^2 for the same heads
+        const int nbs = nb_of(b);
+        const int32_t L = len_of(b);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const double mine0 = (kq < 2) ? cm[m][0] : cs[m][0];
+            const double mine1 = (kq < 2) ? cm[m][1] : cs[m][1];
+            const double oth0 = __shfl_xor_sync(0xffffffffu, mine0, 2);
+            const double oth1 = __shfl_xor_sync(0xffffffffu, mine1, 2);
+            const int j = t * kTile + 8 * m + prow;
+            if (kq < 2 && j < nbs) {
                 const int nj = min(c.bs, L - j * c.bs);
                 // log n_j: a constant except for a sequence's last block
-                double sc = ((nj == c.bs) ? log_bs : log((double)nj)) + tot;
-                if (!first_order) {
-                    // log1p in fp32 where it is accurate to ~6e-8 absolute (argument <= 1)
-                    const double x = 0.5 * t2;
-                    sc += (x <= 1.0) ? (double)log1pf((float)x) : log1p(x);
+                const double lg = (nj == c.bs) ? log_bs : c_log_n[nj];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int g = 2 * kq + e;
+                    if (g < G) {
+                        double sc = lg + (e ? mine1 : mine0);
+                        if (!first_order) {
+                            // fp32 log1p: within one fp32 ulp of the result, under 2.5e-7
+                            // while the argument stays below e^4 - 1
+                            sc += (double)log1pf((float)(0.5 * (e ? oth1 : oth0)));
+                        }
+                        scores[((int64_t)b * c.hq + h * G + g) * c.mbp + j] = (float)sc;
+                    }
                 }
-                scores[((int64_t)b * c.hq + h * G + g) * c.mbp + j] = (float)sc;
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
     }
 }
 
@@ -495,31 +639,37 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
 }
 
 template <int D, typename T>
-static cudaError_t launch_score_t(const CacheView& c, const void* q, double scale, int first_order,
-                                  float* scores, int chunk, float* gread, int32_t* status,
-                                  cudaStream_t s) {
-    const int nchunks = (c.mbp + chunk - 1) / chunk;
-    const size_t ring = (size_t)kScoreStages * kScoreStageBlocks * 2 * D * sizeof(float);
-    const size_t rd = (size_t)(4 * D + kScoreWarps * 4 * (D + 1)) * sizeof(float);
-    const size_t smem = ring > rd ? ring : rd;
+static cudaError_t launch_score_t(const CacheView& c, const CUtensorMap& tstats, const void* q,
+                                  double scale, int first_order, float* scores, float* gread,
+                                  int32_t* status, cudaStream_t s) {
+    using S = ScoreShape<D>;
+    const int groups = c.batch * c.hkv;
+    const int ntile = (c.mbp + kTile - 1) / kTile;
+    const int64_t nitems = (int64_t)groups * (S::kReadoutParts + ntile);
+    const int grid = (int)std::min<int64_t>((nitems + kScoreWarps - 1) / kScoreWarps,
+                                            (int64_t)kScoreCtasPerSm * kNumSms);
     cudaError_t e = cudaFuncSetAttribute(score_kernel<D, T>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(score_kernel<D, T>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    dim3 grid(nchunks + 1, c.batch * c.hkv);
-    return launch_pdl(score_kernel<D, T>, grid, dim3((kScoreWarps + 1) * 32), smem, s, c,
-                      (const T*)q, scale, first_order, scores, chunk, nchunks, gread, status);
+    return launch_pdl(score_kernel<D, T>, dim3(grid), dim3(kScoreWarps * 32), S::kSmem, s, tstats,
+                      c, (const T*)q, scale, log((double)c.bs), first_order, scores, gread, ntile,
+                      status);
 }
 
-cudaError_t launch_score(const CacheView& c, int dtype, const void* q, double scale,
-                         int first_order, float* scores, int chunk, float* gread,
+int score_readout_parts(int d) {
+    return d == 128 ? ScoreShape<128>::kReadoutParts : ScoreShape<64>::kReadoutParts;
+}
+
+cudaError_t launch_score(const CacheView& c, const CUtensorMap& tstats, int dtype, const void* q,
+                         double scale, int first_order, float* scores, float* gread,
                          int32_t* status, cudaStream_t s) {
     if (dtype == SPLA_BF16)
-        return c.d == 128 ? launch_score_t<128, __nv_bfloat16>(c, q, scale, first_order, scores, chunk, gread, status, s)
-                          : launch_score_t<64, __nv_bfloat16>(c, q, scale, first_order, scores, chunk, gread, status, s);
-    return c.d == 128 ? launch_score_t<128, float>(c, q, scale, first_order, scores, chunk, gread, status, s)
-                      : launch_score_t<64, float>(c, q, scale, first_order, scores, chunk, gread, status, s);
+        return c.d == 128 ? launch_score_t<128, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, gread, status, s)
+                          : launch_score_t<64, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, gread, status, s);
+    return c.d == 128 ? launch_score_t<128, float>(c, tstats, q, scale, first_order, scores, gread, status, s)
+                      : launch_score_t<64, float>(c, tstats, q, scale, first_order, scores, gread, status, s);
 }
 
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
