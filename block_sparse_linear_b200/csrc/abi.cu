@@ -13,7 +13,7 @@ cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, cons
                           const int32_t* n_new, int32_t max_new, int32_t* status, cudaStream_t s);
 cudaError_t launch_score(const CacheView& c, const CUtensorMap& tstats, int dtype, const void* q,
                          double scale, int first_order, float* scores, float* gread,
-                         int32_t* status, cudaStream_t s);
+                         float* aw, int32_t* status, cudaStream_t s);
 int score_readout_parts(int d);
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
                           const float* scores, uint32_t* bits, int nw, int32_t* nsel,
@@ -120,6 +120,8 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     off = align256(off + (size_t)groups * ns * G * L.rec * sizeof(float));
     L.off_gread = off;
     off = align256(off + (size_t)groups * L.readout_parts * G * (p->head_dim + 4) * sizeof(float));
+    L.off_aw = off;
+    off = align256(off + (size_t)groups * p->head_dim * 4 * sizeof(float));
     L.total = off;
     return L;
 }
@@ -271,10 +273,11 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
 
     prof_mark(0, s);
     float* gread = reinterpret_cast<float*>(ws + L.off_gread);
+    float* aw_ws = reinterpret_cast<float*>(ws + L.off_aw);
     CUtensorMap tstats;
     if (!make_stats_map(&tstats, v)) return cuda_fail(cudaErrorInvalidValue);
     cudaError_t e = launch_score(v, tstats, params->dtype, q, scale, first_order, scores, gread,
-                                 dev_status, s);
+                                 aw_ws, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(1, s);
     e = launch_select(v, params->top_k, params->n_sink, params->n_local, scores, bits, L.nw, nsel,
@@ -297,6 +300,7 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     da.max_per = L.max_per;
     da.no_rla = no_rla;
     da.nrd = L.readout_parts;
+    da.aw = aw_ws;
     da.sl2 = sl2;
     da.eps = eps;
     if (use_mma) {

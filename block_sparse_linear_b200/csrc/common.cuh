@@ -39,7 +39,7 @@ struct DecodeLayout {
     int32_t rec;             // floats per partial record
     int32_t readout_parts;   // row ranges of S the global readout is split into
     int32_t max_per;         // union blocks one decode CTA may receive
-    size_t off_scores, off_bits, off_nsel, off_part, off_gread, total;
+    size_t off_scores, off_bits, off_nsel, off_part, off_gread, off_aw, total;
 };
 
 // Per-call arguments of the decode kernels beyond the cache.
@@ -53,6 +53,7 @@ struct DecodeArgs {
     const int32_t* nsel;        // [batch][Hq]
     float* part;                // [batch*Hkv][nsplit][G][rec]
     const float* gread;         // [batch*Hkv][nrd][G][d+4]: readout parts, N (d) then D
+    const float* aw;            // [batch*Hkv][d][4] phi weights a_g,i (written by the scoring kernel)
     int32_t* status;
     int nw, nsplit, max_per, no_rla, nrd;
     float sl2, eps;
@@ -91,6 +92,24 @@ template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x
 template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Packed fp32 pair arithmetic (sm_100): one instruction for two lanes of work.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll

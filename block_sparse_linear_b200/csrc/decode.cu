@@ -39,21 +39,48 @@
 namespace spla {
 
 // ------------------------------------------------------------------ shared prologue pieces
-// Union of the G heads' selections, this CTA's share, built by all nthr threads:
-// per-word union popcounts, one warp's exclusive scan, parallel extraction of
-// the share's blocks and head masks, then parallel block-table lookups.
-// wcnt: >= nw ints of scratch. Returns the share's length (all threads).
-__device__ int build_union_share(const CacheView& c, const uint32_t* bits, int nw, int b, int h,
-                                 int nb, int split, int nsplit, int max_per, int32_t* blk,
-                                 int32_t* phys, uint32_t* hm, int* wcnt, int* s_n,
-                                 int32_t* status, int tid, int nthr) {
+// Phase 1, one round of loads by all threads: the G heads' selection bitset
+// words of this group into wbits ([G][nwu], shared memory), and the query-side
+// constants qs[g][i] = q (fp32), ml[i] = m_i * log2e and the phi weights
+// aw[g][i] = exp(q_g,i + m_i - c_g) the scoring kernel wrote for the global
+// readout (the kept blocks' term uses the very same weights).
+// (Out of line, scalar arguments: the prologue does not add to the register
+// pressure of the streaming loop that follows it.)
+__device__ __noinline__ void stage_group(const uint32_t* bits, int nw, const void* q,
+                                         const float* aw_ws, const float* m, int hq, int hkv,
+                                         int G, int d, int is_bf16, int b, int h, int nwu,
+                                         uint32_t* wbits, float* qs, float* ml, float* aw,
+                                         int tid, int nthr) {
+    const int gi = b * hkv + h;
+    const uint32_t* hb = bits + ((int64_t)b * hq + h * G) * nw;
+    for (int e = tid; e < G * nwu; e += nthr) {
+        const int g = e / nwu, w = e % nwu;
+        wbits[e] = __ldcg(hb + (int64_t)g * nw + w);
+    }
+    const float* mrow = m + (int64_t)gi * d;
+    for (int e = tid; e < G * d; e += nthr) {
+        const int g = e / d, i = e % d;
+        const int64_t qi = ((int64_t)b * hq + h * G + g) * d + i;
+        qs[e] = is_bf16 ? __bfloat162float(((const __nv_bfloat16*)q)[qi]) : ((const float*)q)[qi];
+        aw[e] = __ldcg(aw_ws + ((int64_t)gi * d + i) * 4 + g);
+    }
+    for (int i = tid; i < d; i += nthr) ml[i] = mrow[i] * SPLA_LOG2E;
+}
+
+// Phase 2, after a barrier, from shared memory: the union of the G selections
+// (a block read once for all heads that kept it), per-word counts and their
+// prefix sums (one warp), this CTA's equal share [u0, u1) of the union with
+// per-block head masks, then a second round of loads for the share's physical
+// blocks. wcnt: nwu ints of scratch. Returns the share's length (all threads).
+__device__ __noinline__ int union_share(const int32_t* table, int mbp, int num_phys, int G,
+                                        const uint32_t* wbits, int nwu, int nb, int b, int split,
+                                        int nsplit, int max_per, int* wcnt, int32_t* blk,
+                                        int32_t* phys, uint32_t* hm, int* s_n, int32_t* status,
+                                        int tid, int nthr) {
     const int lane = tid & 31, warp = tid >> 5;
-    const int G = c.group;
-    const int nwu = (nb + 31) >> 5;
-    const uint32_t* hb = bits + ((int64_t)b * c.hq + h * G) * nw;
     auto word = [&](int w) -> uint32_t {
         uint32_t u = 0u;
-        for (int g = 0; g < G; ++g) u |= __ldg(hb + (int64_t)g * nw + w);
+        for (int g = 0; g < G; ++g) u |= wbits[g * nwu + w];
         if (w == nwu - 1 && (nb & 31)) u &= (1u << (nb & 31)) - 1u;
         return u;
     };
@@ -77,9 +104,8 @@ __device__ int build_union_share(const CacheView& c, const uint32_t* bits, int n
             run += v;
         }
         if (lane == 31) {
-            const int U = x;
-            s_n[0] = (int)(((int64_t)split * U) / nsplit);          // u0
-            s_n[1] = (int)(((int64_t)(split + 1) * U) / nsplit);    // u1
+            s_n[0] = (int)(((int64_t)split * x) / nsplit);          // u0
+            s_n[1] = (int)(((int64_t)(split + 1) * x) / nsplit);    // u1
         }
     }
     __syncthreads();
@@ -95,7 +121,7 @@ __device__ int build_union_share(const CacheView& c, const uint32_t* bits, int n
             u &= u - 1u;
             if (r >= u0 && r < u1 && r - u0 < max_per) {
                 uint32_t mask = 0u;
-                for (int g = 0; g < G; ++g) mask |= ((__ldg(hb + (int64_t)g * nw + w) >> bit) & 1u) << g;
+                for (int g = 0; g < G; ++g) mask |= ((wbits[g * nwu + w] >> bit) & 1u) << g;
                 blk[r - u0] = (w << 5) + bit;
                 hm[r - u0] = mask;
             }
@@ -105,8 +131,9 @@ __device__ int build_union_share(const CacheView& c, const uint32_t* bits, int n
     __syncthreads();
     const int n = min(u1 - u0, max_per);
     for (int e = tid; e < n; e += nthr) {
-        int32_t p = c.table[(int64_t)b * c.mbp + blk[e]];
-        if (p < 0 || p >= c.num_phys) {
+        int32_t p = table[(int64_t)b * mbp + blk[e]];
+        if (p < 0 || p >= num_phys) {
+            // read nothing from it: no head attends to it
             set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
             p = 0;
             hm[e] = 0u;
@@ -115,42 +142,6 @@ __device__ int build_union_share(const CacheView& c, const uint32_t* bits, int n
     }
     __syncthreads();
     return n;
-}
-
-// Query-side constants, computed by nthr threads (tid in [0, nthr)); the caller
-// synchronises between the three steps:
-//   1) qs[g][i] = q (fp32), ml[i] = m_i * log2e
-//   2) cg[g] = max_i (q_i + m_i)                  (warps 0..G-1)
-//   3) aw[g][i] = exp(q_i + m_i - c_g)
-__device__ void query_load(const CacheView& c, const void* q, int is_bf16, int b, int h,
-                           float* qs, float* ml, int tid, int nthr) {
-    const int G = c.group, d = c.d;
-    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
-    for (int e = tid; e < G * d; e += nthr) {
-        const int g = e / d, i = e % d;
-        const int64_t qi = ((int64_t)b * c.hq + h * G + g) * d + i;
-        qs[e] = is_bf16 ? __bfloat162float(((const __nv_bfloat16*)q)[qi]) : ((const float*)q)[qi];
-    }
-    for (int i = tid; i < d; i += nthr) ml[i] = mrow[i] * SPLA_LOG2E;
-}
-
-__device__ void query_max(const CacheView& c, int b, int h, const float* qs, float* cg, int tid) {
-    const int G = c.group, d = c.d;
-    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
-    const int warp = tid >> 5, lane = tid & 31;
-    if (warp < G) {
-        float mx = -SPLA_INF;
-        for (int i = lane; i < d; i += 32) mx = fmaxf(mx, qs[warp * d + i] + mrow[i]);
-        mx = warp_max(mx);
-        if (lane == 0) cg[warp] = mx;
-    }
-}
-
-__device__ void query_phi(const CacheView& c, int b, int h, const float* qs, const float* cg,
-                          float* aw, int tid, int nthr) {
-    const int G = c.group, d = c.d;
-    const float* mrow = c.m + ((int64_t)b * c.hkv + h) * d;
-    for (int e = tid; e < G * d; e += nthr) aw[e] = expf(qs[e] + mrow[e % d] - cg[e / d]);
 }
 
 // ------------------------------------------------------------------ combine
@@ -290,7 +281,6 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         (reinterpret_cast<uintptr_t>(hm + a.max_per) + 15) & ~uintptr_t(15));   // [4][D]
     float* aw = qs + G4 * D;                                // [4][D]
     float* ml = aw + G4 * D;                                // [D]
-    float* cg = ml + D;                                     // [4]
     __shared__ int s_n[2], s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -316,12 +306,19 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         fence_barrier_init();
         s_abort = 0;
     }
-    // the union share first (all threads; the word counts borrow stage 0, no TMA yet)
-    const int nblk = (nb > 0) ? build_union_share(c, a.bits, a.nw, b, h, nb, split, nsplit,
-                                                  a.max_per, blk, phys, hm,
-                                                  reinterpret_cast<int*>(stages), s_n, a.status,
-                                                  tid, blockDim.x)
-                              : 0;
+    // the group's bitsets and query constants, then this CTA's share of the union
+    // (the bitset words and counts borrow the stage buffers, no TMA in flight yet)
+    const int nwu = (nb + 31) >> 5;
+    uint32_t* wbits = reinterpret_cast<uint32_t*>(stages);
+    int nblk = 0;
+    if (nb > 0) {
+        stage_group(a.bits, a.nw, a.q, a.aw, c.m, c.hq, c.hkv, G, D, 1, b, h, nwu, wbits, qs, ml,
+                    aw, tid, blockDim.x);
+        __syncthreads();
+        nblk = union_share(c.table, c.mbp, c.num_phys, G, wbits, nwu, nb, b, split, nsplit,
+                           a.max_per, reinterpret_cast<int*>(wbits + G * nwu), blk, phys, hm, s_n,
+                           a.status, tid, blockDim.x);
+    }
 
     if (nb == 0) {
         for (int e = tid; e < G * REC; e += blockDim.x) {
@@ -341,7 +338,7 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     if (warp == NCW) {
         // ---------------- producer: TMA ring over 64-token units
         if (lane == 0) {
-            fence_proxy_async();   // stage 0 held the union word counts (generic writes)
+            fence_proxy_async();   // order this CTA's generic shared-memory writes before TMA
             int u = 0;
             for (int it = 0; it < nblk && !s_abort; ++it) {
                 for (int half = 0; half < UPB; ++half) {
@@ -366,14 +363,7 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
             }
         }
     } else {
-        // ---------------- consumers: query constants while the first tiles land
-        query_load(c, a.q, 1, b, h, qs, ml, tid, NCW * 32);
-        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
-        query_max(c, b, h, qs, cg, tid);
-        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
-        query_phi(c, b, h, qs, cg, aw, tid, NCW * 32);
-        asm volatile("bar.sync 1, %0;" :: "r"(NCW * 32));
-        // B fragments: column n = lane/4; rows k = 2*(lane%4) (+1, +8, +9) of each 16-dim step
+        // ---------------- consumers: B fragments while the first tiles land: column n = lane/4; rows k = 2*(lane%4) (+1, +8, +9) of each 16-dim step
         uint32_t qf[D / 16][2], wf[D / 16][2];
         {
             const int n = lane >> 2;
@@ -443,6 +433,7 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
                         const float2 mA = *reinterpret_cast<const float2*>(ml + kb);
                         const float2 mB = *reinterpret_cast<const float2*>(ml + kb + 8);
                         uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+                        // phi = exp(k - m) of a bf16 pair, split into bf16 hi + lo
                         auto phi = [&](uint32_t kr, float m0, float m1, uint32_t& hi, uint32_t& lo) {
                             const float x0 = ex2(fmaf(bf16_lo(kr), SPLA_LOG2E, -m0));
                             const float x1 = ex2(fmaf(bf16_hi(kr), SPLA_LOG2E, -m1));
@@ -494,12 +485,15 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
                     dt_run[0] += w00 + w10;
                     dt_run[1] += w01 + w11;
                     const float g0 = lo_half ? f0 : 1.f, g1 = lo_half ? f1 : 1.f;
+                    // the running maxima rarely move once the first tiles are in
+                    if (!__all_sync(0xffffffffu, g0 == 1.f && g1 == 1.f)) {
 #pragma unroll
-                    for (int mt = 0; mt < D / 16; ++mt) {
-                        acc[mt][0] *= g0;
-                        acc[mt][1] *= g1;
-                        acc[mt][2] *= g0;
-                        acc[mt][3] *= g1;
+                        for (int mt = 0; mt < D / 16; ++mt) {
+                            acc[mt][0] *= g0;
+                            acc[mt][1] *= g1;
+                            acc[mt][2] *= g0;
+                            acc[mt][3] *= g1;
+                        }
                     }
                     // [P | W] as a 16 x 8 matrix in C layout: lanes with cols 4..7 take W from lane-2
                     const float wv[4] = {w00, w01, w10, w11};
@@ -630,15 +624,15 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const Dec
         }
         return;
     }
-    // union share (all threads; the word counts borrow the K tile)
-    const int nblk = build_union_share(c, a.bits, a.nw, b, h, nb, split, nsplit, a.max_per, blk,
-                                       phys, hm, reinterpret_cast<int*>(Ks), s_n, a.status, tid,
-                                       blockDim.x);
-    query_load(c, a.q, sizeof(T) == 2, b, h, qs, ml, tid, blockDim.x);
+    // bitset words and counts borrow the K and V tiles
+    const int nwu = (nb + 31) >> 5;
+    uint32_t* wbits = reinterpret_cast<uint32_t*>(Ks);
+    stage_group(a.bits, a.nw, a.q, a.aw, c.m, c.hq, c.hkv, G, d, sizeof(T) == 2, b, h, nwu, wbits,
+                qs, ml, aw, tid, blockDim.x);
     __syncthreads();
-    query_max(c, b, h, qs, cg, tid);
-    __syncthreads();
-    query_phi(c, b, h, qs, cg, aw, tid, blockDim.x);
+    const int nblk = union_share(c.table, c.mbp, c.num_phys, G, wbits, nwu, nb, b, split, nsplit,
+                                 a.max_per, reinterpret_cast<int*>(wbits + G * nwu), blk, phys, hm,
+                                 s_n, a.status, tid, blockDim.x);
     if (tid < 4) { s_m[tid] = -SPLA_INF; s_l[tid] = 0.f; s_dt[tid] = 0.f; }
     __syncthreads();
     // accumulators: thread owns (g, j) pairs e = tid + 256*u

@@ -106,7 +106,7 @@ template <int D, typename T>
 __global__ void __launch_bounds__(kScoreWarps * 32, kScoreCtasPerSm)
 score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* __restrict__ q,
              double scale, double log_bs, int first_order, float* __restrict__ scores,
-             float* __restrict__ gread, int ntile, int32_t* status) {
+             float* __restrict__ gread, float* __restrict__ aw_out, int ntile, int32_t* status) {
     using S = ScoreShape<D>;
     constexpr int RP = S::kReadoutParts, TS = S::kTileStages, RPS = S::kRowsPerStage;
     constexpr int CPL = D / 32;                    // readout columns per lane
@@ -266,6 +266,11 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
                 }
             }
             __syncwarp();
+            if (part == 0) {
+                // the decode kernels weight phi(k) with the same a_g,i
+                float4* awg = reinterpret_cast<float4*>(aw_out + (int64_t)gi * D * 4);
+                for (int r = lane; r < D; r += 32) awg[r] = *reinterpret_cast<const float4*>(at + r * 4);
+            }
             float acc[4][CPL];
 #pragma unroll
             for (int g = 0; g < 4; ++g)
@@ -440,6 +445,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
     __shared__ int wpre[SPLA_MAX_BLOCKS_PER_SEQ / 32];             // per-word counts, then prefixes
     __shared__ uint32_t cand_key[kCandCap];
     __shared__ int cand_idx[kCandCap];
+    __shared__ __align__(16) unsigned long long cand_c[kCandCap];   // key << 32 | ~index
     __shared__ int tmp[40];
     __shared__ unsigned long long s_lo, s_hi;
     __shared__ int s_krem, s_cnt, s_done, s_mode, s_ncand, s_total;
@@ -561,11 +567,26 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
             }
             __syncthreads();
             const int nc = min(s_ncand, kCandCap);
+            // one composite per candidate: a larger key, or an equal key at a lower
+            // block index, compares greater
+            const int ncp = (nc + 7) & ~7;
+            for (int i = tid; i < ncp; i += kSelThreads)
+                cand_c[i] = (i < nc) ? (((unsigned long long)cand_key[i] << 32) |
+                                        (uint32_t)~(uint32_t)cand_idx[i])
+                                     : 0ull;
+            __syncthreads();
             for (int i = tid; i < nc; i += kSelThreads) {
+                const unsigned long long mine = cand_c[i];
                 int rank = 0;
-                for (int o = 0; o < nc; ++o)
-                    rank += (cand_key[o] > cand_key[i]) ||
-                            (cand_key[o] == cand_key[i] && cand_idx[o] < cand_idx[i]);
+                // eight candidates per step, their loads in flight together
+                for (int o = 0; o < ncp; o += 8) {
+                    const ulonglong2 x0 = *reinterpret_cast<const ulonglong2*>(cand_c + o);
+                    const ulonglong2 x1 = *reinterpret_cast<const ulonglong2*>(cand_c + o + 2);
+                    const ulonglong2 x2 = *reinterpret_cast<const ulonglong2*>(cand_c + o + 4);
+                    const ulonglong2 x3 = *reinterpret_cast<const ulonglong2*>(cand_c + o + 6);
+                    rank += (x0.x > mine) + (x0.y > mine) + (x1.x > mine) + (x1.y > mine) +
+                            (x2.x > mine) + (x2.y > mine) + (x3.x > mine) + (x3.y > mine);
+                }
                 if (rank < krem) keys[cand_idx[i]] = 0xffffffffu;
             }
         } else {
@@ -641,7 +662,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
 template <int D, typename T>
 static cudaError_t launch_score_t(const CacheView& c, const CUtensorMap& tstats, const void* q,
                                   double scale, int first_order, float* scores, float* gread,
-                                  int32_t* status, cudaStream_t s) {
+                                  float* aw, int32_t* status, cudaStream_t s) {
     using S = ScoreShape<D>;
     const int groups = c.batch * c.hkv;
     const int ntile = (c.mbp + kTile - 1) / kTile;
@@ -654,8 +675,8 @@ static cudaError_t launch_score_t(const CacheView& c, const CUtensorMap& tstats,
     e = cudaFuncSetAttribute(score_kernel<D, T>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     return launch_pdl(score_kernel<D, T>, dim3(grid), dim3(kScoreWarps * 32), S::kSmem, s, tstats,
-                      c, (const T*)q, scale, log((double)c.bs), first_order, scores, gread, ntile,
-                      status);
+                      c, (const T*)q, scale, log((double)c.bs), first_order, scores, gread, aw,
+                      ntile, status);
 }
 
 int score_readout_parts(int d) {
@@ -664,23 +685,22 @@ int score_readout_parts(int d) {
 
 cudaError_t launch_score(const CacheView& c, const CUtensorMap& tstats, int dtype, const void* q,
                          double scale, int first_order, float* scores, float* gread,
-                         int32_t* status, cudaStream_t s) {
+                         float* aw, int32_t* status, cudaStream_t s) {
     if (dtype == SPLA_BF16)
-        return c.d == 128 ? launch_score_t<128, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, gread, status, s)
-                          : launch_score_t<64, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, gread, status, s);
-    return c.d == 128 ? launch_score_t<128, float>(c, tstats, q, scale, first_order, scores, gread, status, s)
-                      : launch_score_t<64, float>(c, tstats, q, scale, first_order, scores, gread, status, s);
+        return c.d == 128 ? launch_score_t<128, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, gread, aw, status, s)
+                          : launch_score_t<64, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, gread, aw, status, s);
+    return c.d == 128 ? launch_score_t<128, float>(c, tstats, q, scale, first_order, scores, gread, aw, status, s)
+                      : launch_score_t<64, float>(c, tstats, q, scale, first_order, scores, gread, aw, status, s);
 }
 
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
                           const float* scores, uint32_t* bits, int nw, int32_t* nsel,
                           int32_t* sel_idx, int kcap, cudaStream_t s) {
     const size_t smem = (size_t)((c.mbp + 31) / 32) * 32 * sizeof(uint32_t);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(select_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
+    // static plus dynamic shared memory may pass the 48 KiB default
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
     return launch_pdl(select_kernel, dim3(c.batch * c.hq), dim3(kSelThreads), smem, s, c, top_k,
                       n_sink, n_local, scores, bits, nw, nsel, sel_idx, kcap);
 }
