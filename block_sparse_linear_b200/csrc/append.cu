@@ -4,15 +4,16 @@
 // mean and diagonal variance, section 2.2 for the global state that linear
 // attention over all blocks reads, section 2.3 for the feature map exp).
 //
-// Three launches, stream-ordered:
-//   append_kv_stats  grid (touched blocks, batch*Hkv): write tokens, then the
-//                    block's mean and population variance in fp64 (two-pass,
-//                    keys staged in shared memory);
-//   append_state     grid (d/8 row groups, batch*Hkv): m <- max(m, k_new),
-//                    rescale S and z rows by exp(m_old - m_new), add
-//                    exp(k - m_new) v^T and exp(k - m_new);
+// Two launches, stream-ordered:
+//   append_kernel    grid (touched blocks + d/8 row groups, batch*Hkv), two
+//                    independent roles that both read the old context_lens:
+//                    CTAs x < nsb write the tokens of logical block
+//                    L0/B + x, then its mean and population variance in fp64
+//                    (two-pass, keys staged in shared memory); the other CTAs
+//                    own 8 rows of S (and of z, m): m <- max(m, k_new), rescale
+//                    by exp(m_old - m_new), add exp(k - m_new) v^T and
+//                    exp(k - m_new);
 //   append_advance   one CTA: context_lens[b] += n_new[b].
-// The first two read the old context_lens and are independent of each other.
 #include "common.cuh"
 
 namespace spla {
@@ -29,24 +30,20 @@ __device__ __forceinline__ bool append_ok(const CacheView& c, const int32_t* n_n
     return true;
 }
 
+// Tokens and statistics of logical block L0/B + x of one (sequence, KV head).
 template <typename T>
-__global__ void __launch_bounds__(256) append_kv_stats_kernel(CacheView c, const T* k_new,
-                                                              const T* v_new,
-                                                              const int32_t* n_new,
-                                                              int32_t max_new, int32_t* status) {
-    const int b = blockIdx.y / c.hkv;
-    const int h = blockIdx.y % c.hkv;
-    pdl_trigger();
-    pdl_wait();
+__device__ void append_block(const CacheView& c, const T* k_new, const T* v_new,
+                             const int32_t* n_new, int32_t max_new, int32_t* status, int b, int h,
+                             int x, float* ktile) {
     int32_t L0, n;
     if (!append_ok(c, n_new, max_new, b, &L0, &n)) {
-        if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0)
+        if (x == 0 && h == 0 && threadIdx.x == 0)
             set_status(status, (n < 0 || n > max_new) ? SPLA_DEV_BAD_COUNT : SPLA_DEV_CAPACITY);
         return;
     }
     if (n == 0) return;
     const int bs = c.bs, d = c.d;
-    const int lb = L0 / bs + blockIdx.x;            // logical block this CTA owns
+    const int lb = L0 / bs + x;                     // logical block this CTA owns
     const int64_t blk_lo = (int64_t)lb * bs;
     if (blk_lo >= (int64_t)L0 + n) return;
     const int32_t phys = c.table[(int64_t)b * c.mbp + lb];
@@ -69,7 +66,6 @@ __global__ void __launch_bounds__(256) append_kv_stats_kernel(CacheView c, const
     __syncthreads();
     // statistics over all tokens now in the block: stage the keys in shared
     // memory with coalesced loads, then two passes per dimension in fp64
-    extern __shared__ float ktile[];                 // [nj][d]
     const int nj = t_end - (int)blk_lo;
     for (int e = threadIdx.x; e < nj * d; e += blockDim.x) ktile[e] = to_f(kp[e]);
     __syncthreads();
@@ -100,21 +96,16 @@ __global__ void __launch_bounds__(256) append_kv_stats_kernel(CacheView c, const
     }
 }
 
-// Rows [8*blockIdx.x, +8) of S (and the same entries of z, m) of one (sequence, KV head).
+// Rows [8*rg, +8) of S (and the same entries of z, m) of one (sequence, KV head).
 // Warp r owns row r; lane l owns columns l, l+32, ... of that row.
 template <typename T>
-__global__ void __launch_bounds__(256) append_state_kernel(CacheView c, const T* k_new,
-                                                           const T* v_new, const int32_t* n_new,
-                                                           int32_t max_new) {
-    const int b = blockIdx.y / c.hkv;
-    const int h = blockIdx.y % c.hkv;
-    pdl_trigger();
-    pdl_wait();
+__device__ void append_rows(const CacheView& c, const T* k_new, const T* v_new,
+                            const int32_t* n_new, int32_t max_new, int b, int h, int rg) {
     int32_t L0, n;
     if (!append_ok(c, n_new, max_new, b, &L0, &n) || n == 0) return;
     const int d = c.d;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row = blockIdx.x * 8 + warp;
+    const int row = rg * 8 + warp;
     if (row >= d) return;
     const int64_t gidx = ((int64_t)b * c.hkv + h) * d + row;
     float* Srow = c.S + gidx * d;
@@ -165,6 +156,22 @@ __global__ void __launch_bounds__(256) append_state_kernel(CacheView c, const T*
     }
 }
 
+// One launch for both roles: CTAs x < nsb take blocks, the rest take row groups.
+template <typename T>
+__global__ void __launch_bounds__(256) append_kernel(CacheView c, const T* k_new, const T* v_new,
+                                                     const int32_t* n_new, int32_t max_new,
+                                                     int nsb, int32_t* status) {
+    extern __shared__ float ktile[];                 // [B][d], block role only
+    const int b = blockIdx.y / c.hkv;
+    const int h = blockIdx.y % c.hkv;
+    pdl_trigger();
+    pdl_wait();
+    if ((int)blockIdx.x < nsb)
+        append_block<T>(c, k_new, v_new, n_new, max_new, status, b, h, blockIdx.x, ktile);
+    else
+        append_rows<T>(c, k_new, v_new, n_new, max_new, b, h, blockIdx.x - nsb);
+}
+
 __global__ void append_advance_kernel(CacheView c, const int32_t* n_new, int32_t max_new) {
     pdl_trigger();
     pdl_wait();
@@ -198,31 +205,22 @@ cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, cons
                           const int32_t* n_new, int32_t max_new, int32_t* status,
                           cudaStream_t s) {
     if (max_new > 0) {
-        dim3 g1((max_new + c.bs - 1) / c.bs + 1, c.batch * c.hkv);
-        dim3 g2((c.d + 7) / 8, c.batch * c.hkv);
+        const int nsb = (max_new + c.bs - 1) / c.bs + 1;     // blocks a sequence's tokens can touch
+        dim3 grid(nsb + (c.d + 7) / 8, c.batch * c.hkv);
         const size_t smem = (size_t)c.bs * c.d * sizeof(float);
-        if (smem > 48 * 1024) {
-            cudaError_t e = dtype == SPLA_BF16
-                ? cudaFuncSetAttribute(append_kv_stats_kernel<__nv_bfloat16>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                : cudaFuncSetAttribute(append_kv_stats_kernel<float>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-        }
-        cudaError_t e;
+        cudaError_t e = dtype == SPLA_BF16
+            ? cudaFuncSetAttribute(append_kernel<__nv_bfloat16>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+            : cudaFuncSetAttribute(append_kernel<float>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
         if (dtype == SPLA_BF16) {
             using B16 = __nv_bfloat16;
-            e = launch_pdl(append_kv_stats_kernel<B16>, g1, dim3(256), smem, s, c,
-                           (const B16*)k_new, (const B16*)v_new, n_new, max_new, status);
-            if (e == cudaSuccess)
-                e = launch_pdl(append_state_kernel<B16>, g2, dim3(256), 0, s, c, (const B16*)k_new,
-                               (const B16*)v_new, n_new, max_new);
+            e = launch_pdl(append_kernel<B16>, grid, dim3(256), smem, s, c, (const B16*)k_new,
+                           (const B16*)v_new, n_new, max_new, nsb, status);
         } else {
-            e = launch_pdl(append_kv_stats_kernel<float>, g1, dim3(256), smem, s, c,
-                           (const float*)k_new, (const float*)v_new, n_new, max_new, status);
-            if (e == cudaSuccess)
-                e = launch_pdl(append_state_kernel<float>, g2, dim3(256), 0, s, c,
-                               (const float*)k_new, (const float*)v_new, n_new, max_new);
+            e = launch_pdl(append_kernel<float>, grid, dim3(256), smem, s, c, (const float*)k_new,
+                           (const float*)v_new, n_new, max_new, nsb, status);
         }
         if (e != cudaSuccess) return e;
     }

@@ -39,24 +39,18 @@
 namespace spla {
 
 // ------------------------------------------------------------------ shared prologue pieces
-// Phase 1, one round of loads by all threads: the G heads' selection bitset
-// words of this group into wbits ([G][nwu], shared memory), and the query-side
-// constants qs[g][i] = q (fp32), ml[i] = m_i * log2e and the phi weights
-// aw[g][i] = exp(q_g,i + m_i - c_g) the scoring kernel wrote for the global
-// readout (the kept blocks' term uses the very same weights).
+// Query-side constants, loaded before the dependency wait (inputs and what the
+// append and scoring kernels wrote): qs[g][i] = q (fp32), ml[i] = m_i * log2e
+// and the phi weights aw[g][i] = exp(q_g,i + m_i - c_g) the scoring kernel used
+// for the global readout (the kept blocks' term uses the very same weights).
+// With trow non-null, also the sequence's block-table row (mbp entries).
 // (Out of line, scalar arguments: the prologue does not add to the register
 // pressure of the streaming loop that follows it.)
-__device__ __noinline__ void stage_group(const uint32_t* bits, int nw, const void* q,
-                                         const float* aw_ws, const float* m, int hq, int hkv,
-                                         int G, int d, int is_bf16, int b, int h, int nwu,
-                                         uint32_t* wbits, float* qs, float* ml, float* aw,
-                                         int tid, int nthr) {
+__device__ __noinline__ void stage_query(const void* q, const float* aw_ws, const float* m,
+                                         const int32_t* table, int mbp, int hq, int hkv, int G,
+                                         int d, int is_bf16, int b, int h, float* qs, float* ml,
+                                         float* aw, int32_t* trow, int tid, int nthr) {
     const int gi = b * hkv + h;
-    const uint32_t* hb = bits + ((int64_t)b * hq + h * G) * nw;
-    for (int e = tid; e < G * nwu; e += nthr) {
-        const int g = e / nwu, w = e % nwu;
-        wbits[e] = __ldcg(hb + (int64_t)g * nw + w);
-    }
     const float* mrow = m + (int64_t)gi * d;
     for (int e = tid; e < G * d; e += nthr) {
         const int g = e / d, i = e % d;
@@ -65,15 +59,31 @@ __device__ __noinline__ void stage_group(const uint32_t* bits, int nw, const voi
         aw[e] = __ldcg(aw_ws + ((int64_t)gi * d + i) * 4 + g);
     }
     for (int i = tid; i < d; i += nthr) ml[i] = mrow[i] * SPLA_LOG2E;
+    if (trow) {
+        const int32_t* src = table + (int64_t)b * mbp;
+        for (int j = tid; j < mbp; j += nthr) trow[j] = __ldcg(src + j);
+    }
 }
 
-// Phase 2, after a barrier, from shared memory: the union of the G selections
-// (a block read once for all heads that kept it), per-word counts and their
-// prefix sums (one warp), this CTA's equal share [u0, u1) of the union with
-// per-block head masks, then a second round of loads for the share's physical
-// blocks. wcnt: nwu ints of scratch. Returns the share's length (all threads).
-__device__ __noinline__ int union_share(const int32_t* table, int mbp, int num_phys, int G,
-                                        const uint32_t* wbits, int nwu, int nb, int b, int split,
+// After the wait, one round of loads: the G heads' selection bitset words of
+// this group into wbits ([G][nwu], shared memory).
+__device__ __noinline__ void stage_bits(const uint32_t* bits, int nw, int hq, int G, int b, int h,
+                                        int nwu, uint32_t* wbits, int tid, int nthr) {
+    const uint32_t* hb = bits + ((int64_t)b * hq + h * G) * nw;
+    for (int e = tid; e < G * nwu; e += nthr) {
+        const int g = e / nwu, w = e % nwu;
+        wbits[e] = __ldcg(hb + (int64_t)g * nw + w);
+    }
+}
+
+// Then, from shared memory: the union of the G selections (a block read once
+// for all heads that kept it), per-word counts and their prefix sums (one
+// warp), this CTA's equal share [u0, u1) of the union with per-block head
+// masks, and the share's physical blocks from the table row trow (shared or
+// global memory). wcnt: nwu ints of scratch. Returns the share's length (all
+// threads).
+__device__ __noinline__ int union_share(const int32_t* trow, int num_phys, int G,
+                                        const uint32_t* wbits, int nwu, int nb, int split,
                                         int nsplit, int max_per, int* wcnt, int32_t* blk,
                                         int32_t* phys, uint32_t* hm, int* s_n, int32_t* status,
                                         int tid, int nthr) {
@@ -131,7 +141,7 @@ __device__ __noinline__ int union_share(const int32_t* table, int mbp, int num_p
     __syncthreads();
     const int n = min(u1 - u0, max_per);
     for (int e = tid; e < n; e += nthr) {
-        int32_t p = table[(int64_t)b * mbp + blk[e]];
+        int32_t p = trow[blk[e]];
         if (p < 0 || p >= num_phys) {
             // read nothing from it: no head attends to it
             set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
@@ -291,13 +301,15 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
     }
-    pdl_wait();
+    // Before the dependency wait (the selection kernel launches this one once the
+    // scoring kernel has completed): lengths, query constants and the block-table
+    // row, which depend only on the append and scoring kernels. The bitset words,
+    // counts and table row borrow the stage buffers (no TMA in flight yet).
     int32_t L = c.lens[b];
     if (L < 0 || L > c.mbp * c.bs) L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + BS - 1) / BS;
     const int64_t rec_base = (((int64_t)b * c.hkv + h) * nsplit + split) * G;
     constexpr int REC = 2 * D + 4;
-
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -306,18 +318,25 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         fence_barrier_init();
         s_abort = 0;
     }
-    // the group's bitsets and query constants, then this CTA's share of the union
-    // (the bitset words and counts borrow the stage buffers, no TMA in flight yet)
     const int nwu = (nb + 31) >> 5;
     uint32_t* wbits = reinterpret_cast<uint32_t*>(stages);
+    const int trow_off = ((G + 1) * nwu + 3) & ~3;
+    int32_t* trow = reinterpret_cast<int32_t*>(wbits + trow_off);
+    const bool trow_smem = (size_t)(trow_off + c.mbp) * 4 <= (size_t)STAGES * Cfg::STAGE_BYTES;
+    stage_query(a.q, a.aw, c.m, c.table, c.mbp, c.hq, c.hkv, G, D, 1, b, h, qs, ml, aw,
+                (nb > 0 && trow_smem) ? trow : nullptr, tid, blockDim.x);
+    pdl_wait();
+    // the group's selections, then this CTA's share of their union
     int nblk = 0;
     if (nb > 0) {
-        stage_group(a.bits, a.nw, a.q, a.aw, c.m, c.hq, c.hkv, G, D, 1, b, h, nwu, wbits, qs, ml,
-                    aw, tid, blockDim.x);
+        stage_bits(a.bits, a.nw, c.hq, G, b, h, nwu, wbits, tid, blockDim.x);
         __syncthreads();
-        nblk = union_share(c.table, c.mbp, c.num_phys, G, wbits, nwu, nb, b, split, nsplit,
-                           a.max_per, reinterpret_cast<int*>(wbits + G * nwu), blk, phys, hm, s_n,
-                           a.status, tid, blockDim.x);
+        nblk = union_share(trow_smem ? trow : c.table + (int64_t)b * c.mbp, c.num_phys, G, wbits,
+                           nwu, nb, split, nsplit, a.max_per,
+                           reinterpret_cast<int*>(wbits + G * nwu), blk, phys, hm, s_n, a.status,
+                           tid, blockDim.x);
+    } else {
+        __syncthreads();
     }
 
     if (nb == 0) {
@@ -611,7 +630,6 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const Dec
     const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv, split = blockIdx.x;
     const int nsplit = a.nsplit;
     pdl_trigger();
-    pdl_wait();
     int32_t L = c.lens[b];
     if (L < 0 || L > c.mbp * c.bs) L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + BS - 1) / BS;
@@ -627,12 +645,14 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const Dec
     // bitset words and counts borrow the K and V tiles
     const int nwu = (nb + 31) >> 5;
     uint32_t* wbits = reinterpret_cast<uint32_t*>(Ks);
-    stage_group(a.bits, a.nw, a.q, a.aw, c.m, c.hq, c.hkv, G, d, sizeof(T) == 2, b, h, nwu, wbits,
-                qs, ml, aw, tid, blockDim.x);
+    stage_query(a.q, a.aw, c.m, c.table, c.mbp, c.hq, c.hkv, G, d, sizeof(T) == 2, b, h, qs, ml,
+                aw, nullptr, tid, blockDim.x);
+    pdl_wait();
+    stage_bits(a.bits, a.nw, c.hq, G, b, h, nwu, wbits, tid, blockDim.x);
     __syncthreads();
-    const int nblk = union_share(c.table, c.mbp, c.num_phys, G, wbits, nwu, nb, b, split, nsplit,
-                                 a.max_per, reinterpret_cast<int*>(wbits + G * nwu), blk, phys, hm,
-                                 s_n, a.status, tid, blockDim.x);
+    const int nblk = union_share(c.table + (int64_t)b * c.mbp, c.num_phys, G, wbits, nwu, nb,
+                                 split, nsplit, a.max_per, reinterpret_cast<int*>(wbits + G * nwu),
+                                 blk, phys, hm, s_n, a.status, tid, blockDim.x);
     if (tid < 4) { s_m[tid] = -SPLA_INF; s_l[tid] = 0.f; s_dt[tid] = 0.f; }
     __syncthreads();
     // accumulators: thread owns (g, j) pairs e = tid + 256*u

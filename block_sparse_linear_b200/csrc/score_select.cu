@@ -453,8 +453,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
 
     const int b = blockIdx.x / c.hq, hq = blockIdx.x % c.hq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    pdl_trigger();
     pdl_wait();
+    // the decode kernels launch only now: before their own wait they may read what
+    // the scoring kernel wrote (it has completed)
+    pdl_trigger();
     int32_t L = c.lens[b];
     L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + c.bs - 1) / c.bs;
