@@ -2,8 +2,8 @@
 """SPLA decode benchmark on B200: queries*heads/s and achieved HBM bandwidth.
 
 One step = the whole hot path for one batch: spla_append_kv (one new token
-per sequence, updating block statistics and the linear-attention state) then
-spla_decode (score every block -> select top-k -> exact attention over the
+per sequence, updating block statistics and the linear-attention state; two
+launches) then spla_decode (four launches) (score every block -> select top-k -> exact attention over the
 kept blocks with the fused residual-linear-attention term -> combine).
 
 Default workload: batch 4, 32 query / 8 KV heads, d 128, 131072-token
@@ -342,8 +342,8 @@ def run_ours(args):
             "kernels_ms": {n: round(float(np.mean(kt[:, j])), 5) for j, n in enumerate(kernel_names)},
             "kernel_share": {n: round(float(share[j]), 4) for j, n in enumerate(kernel_names)},
             "clocks": clk.summary(),
-            # per step: 3 append kernels + score, select, decode, combine
-            "gpu_launches": 7 * K,
+            # per step: append, length advance, score, select, decode, combine
+            "gpu_launches": 6 * K,
             "dev_status": status,
         }
         if e2e is not None:
