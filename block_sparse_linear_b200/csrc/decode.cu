@@ -67,8 +67,8 @@ __device__ __noinline__ void stage_query(const void* q, const float* aw_ws, cons
 
 // After the wait, one round of loads: the G heads' selection bitset words of
 // this group into wbits ([G][nwu], shared memory).
-__device__ __noinline__ void stage_bits(const uint32_t* bits, int nw, int hq, int G, int b, int h,
-                                        int nwu, uint32_t* wbits, int tid, int nthr) {
+__device__ __forceinline__ void stage_bits(const uint32_t* bits, int nw, int hq, int G, int b,
+                                           int h, int nwu, uint32_t* wbits, int tid, int nthr) {
     const uint32_t* hb = bits + ((int64_t)b * hq + h * G) * nw;
     for (int e = tid; e < G * nwu; e += nthr) {
         const int g = e / nwu, w = e % nwu;
@@ -152,6 +152,71 @@ __device__ __noinline__ int union_share(const int32_t* trow, int num_phys, int G
     }
     __syncthreads();
     return n;
+}
+
+// The same share built by one warp, 32 words at a time (lane l takes word
+// w0 + l): a first sweep counts the union, a second places every word by a
+// shuffle scan and each lane extracts its own word's blocks, head masks and
+// physical blocks. No CTA barrier inside, and no lane walks more than one word
+// per sweep step.
+__device__ __forceinline__ int union_share_warp(const int32_t* trow, int num_phys, int G,
+                                                const uint32_t* wbits, int nwu, int nb, int split,
+                                                int nsplit, int max_per, int32_t* blk,
+                                                int32_t* phys, uint32_t* hm, int32_t* status,
+                                                int lane) {
+    auto word = [&](int w) -> uint32_t {
+        uint32_t u = 0u;
+        for (int g = 0; g < G; ++g) u |= wbits[g * nwu + w];
+        if (w == nwu - 1 && (nb & 31)) u &= (1u << (nb & 31)) - 1u;
+        return u;
+    };
+    int tot = 0;
+    for (int w0 = 0; w0 < nwu; w0 += 32) {
+        const int w = w0 + lane;
+        if (w < nwu) tot += __popc(word(w));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    // the union holds at most 32768 blocks and nsplit is at most 512: 32-bit products
+    const int u0 = split * tot / nsplit, u1 = (split + 1) * tot / nsplit;
+    int base = 0;
+    for (int w0 = 0; w0 < nwu && base < u1; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t u = (w < nwu) ? word(w) : 0u;
+        const int cnt = __popc(u);
+        int x = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        int r = base + x - cnt;
+        base += __shfl_sync(0xffffffffu, x, 31);
+        if (r < u1 && r + cnt > u0) {
+            while (u) {
+                const int bit = __ffs(u) - 1;
+                u &= u - 1u;
+                if (r >= u0 && r < u1 && r - u0 < max_per) {
+                    const int e = r - u0, j = (w << 5) + bit;
+                    uint32_t mask = 0u;
+                    for (int g = 0; g < G; ++g) mask |= ((wbits[g * nwu + w] >> bit) & 1u) << g;
+                    int32_t p = trow[j];
+                    if (p < 0 || p >= num_phys) {
+                        // read nothing from it: no head attends to it
+                        set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
+                        p = 0;
+                        mask = 0u;
+                    }
+                    blk[e] = j;
+                    hm[e] = mask;
+                    phys[e] = p;
+                }
+                ++r;
+            }
+        }
+    }
+    __syncwarp();
+    return min(u1 - u0, max_per);
 }
 
 // ------------------------------------------------------------------ combine
@@ -325,19 +390,47 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     const bool trow_smem = (size_t)(trow_off + c.mbp) * 4 <= (size_t)STAGES * Cfg::STAGE_BYTES;
     stage_query(a.q, a.aw, c.m, c.table, c.mbp, c.hq, c.hkv, G, D, 1, b, h, qs, ml, aw,
                 (nb > 0 && trow_smem) ? trow : nullptr, tid, blockDim.x);
+    __syncthreads();
+    // consumers' B fragments, still before the wait: column n = lane/4; rows
+    // k = 2*(lane%4) (+1, +8, +9) of each 16-dim step
+    uint32_t qf[D / 16][2], wf[D / 16][2];
+    if (warp < NCW) {
+        const int n = lane >> 2;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int kb = kk * 16 + 2 * (lane & 3);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int i = kb + 8 * half;
+                qf[kk][half] = (n < G) ? pack_bf16(qs[n * D + i], qs[n * D + i + 1]) : 0u;
+                uint32_t wv = 0u;
+                const int g = n & 3;
+                if (g < G) {
+                    const float x0 = aw[g * D + i], x1 = aw[g * D + i + 1];
+                    const uint32_t hi = pack_bf16(x0, x1);
+                    wv = (n < 4) ? hi : pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
+                }
+                wf[kk][half] = wv;
+            }
+        }
+    }
     pdl_wait();
-    // the group's selections, then this CTA's share of their union
-    int nblk = 0;
+    // the group's selections (one round of loads by every thread), then the producer
+    // warp alone builds this CTA's share of their union
     if (nb > 0) {
         stage_bits(a.bits, a.nw, c.hq, G, b, h, nwu, wbits, tid, blockDim.x);
         __syncthreads();
-        nblk = union_share(trow_smem ? trow : c.table + (int64_t)b * c.mbp, c.num_phys, G, wbits,
-                           nwu, nb, split, nsplit, a.max_per,
-                           reinterpret_cast<int*>(wbits + G * nwu), blk, phys, hm, s_n, a.status,
-                           tid, blockDim.x);
-    } else {
-        __syncthreads();
+        if (warp == NCW) {
+            const int n = union_share_warp(trow_smem ? trow : c.table + (int64_t)b * c.mbp,
+                                           c.num_phys, G, wbits, nwu, nb, split, nsplit,
+                                           a.max_per, blk, phys, hm, a.status, lane);
+            if (lane == 0) s_n[0] = n;
+        }
+    } else if (tid == 0) {
+        s_n[0] = 0;
     }
+    __syncthreads();
+    const int nblk = s_n[0];
 
     if (nb == 0) {
         for (int e = tid; e < G * REC; e += blockDim.x) {
@@ -382,28 +475,7 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
             }
         }
     } else {
-        // ---------------- consumers: B fragments while the first tiles land: column n = lane/4; rows k = 2*(lane%4) (+1, +8, +9) of each 16-dim step
-        uint32_t qf[D / 16][2], wf[D / 16][2];
-        {
-            const int n = lane >> 2;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const int kb = kk * 16 + 2 * (lane & 3);
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int i = kb + 8 * half;
-                    qf[kk][half] = (n < G) ? pack_bf16(qs[n * D + i], qs[n * D + i + 1]) : 0u;
-                    uint32_t wv = 0u;
-                    const int g = n & 3;
-                    if (g < G) {
-                        const float x0 = aw[g * D + i], x1 = aw[g * D + i + 1];
-                        const uint32_t hi = pack_bf16(x0, x1);
-                        wv = (n < 4) ? hi : pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
-                    }
-                    wf[kk][half] = wv;
-                }
-            }
-        }
+        // ---------------- consumers
         const bool lo_half = (lane & 3) < 2;
         const int qm = lane >> 3, rr = lane & 7;
         const int t0 = warp * 16;                       // this warp's slab of every unit
@@ -557,8 +629,11 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     float* mw = reinterpret_cast<float*>(stages);           // [NCW][4]
     float* lw = mw + NCW * 4;
     float* dw = lw + NCW * 4;
-    float* ap = dw + NCW * 4;                               // [NCW][4][D]
-    float* an = ap + NCW * 4 * D;                           // [NCW][4][D]
+    // per-warp partial rows [NCW][4][D + 4]; the N~ rows start 16 floats further so
+    // that the four lanes writing one column hit four different bank groups
+    constexpr int RP = D + 4;
+    float* ap = dw + NCW * 4;                               // 16-byte aligned (48 floats in)
+    float* an = ap + NCW * 4 * RP + 16;
     if (warp < NCW) {
         if (lane < 2) {
             mw[warp * 4 + c0] = m_run[0];
@@ -574,33 +649,32 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
             for (int r = 0; r < 4; ++r) {
                 const int j = mt * 16 + (lane >> 2) + ((r >> 1) << 3);
                 const int col = 2 * (lane & 3) + (r & 1);
-                float* dst = (col < 4) ? ap + (warp * 4 + col) * D : an + (warp * 4 + col - 4) * D;
+                float* dst = (col < 4) ? ap + (warp * 4 + col) * RP : an + (warp * 4 + col - 4) * RP;
                 dst[j] = acc[mt][r];
             }
     }
     __syncthreads();
-    // merge the consumer warps and write the partial records
-    for (int e = tid; e < G * D; e += blockDim.x) {
-        const int g = e / D, j = e % D;
+    // merge the consumer warps and write the partial records, four columns a thread
+    for (int e = tid; e < G * (D / 4); e += blockDim.x) {
+        const int g = e / (D / 4), j = 4 * (e % (D / 4));
         float M = -SPLA_INF;
         for (int w = 0; w < NCW; ++w) M = fmaxf(M, mw[w * 4 + g]);
-        float l = 0.f, o = 0.f, nt = 0.f, dt = 0.f;
+        float l = 0.f, dt = 0.f;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f), nt = o;
+#pragma unroll
         for (int w = 0; w < NCW; ++w) {
             const float f = (M == -SPLA_INF) ? 0.f : ex2(mw[w * 4 + g] - M);
             l += lw[w * 4 + g] * f;
-            o += ap[(w * 4 + g) * D + j] * f;
-            nt += an[(w * 4 + g) * D + j];
             dt += dw[w * 4 + g];
+            const float4 pa = *reinterpret_cast<const float4*>(ap + (w * 4 + g) * RP + j);
+            const float4 pn = *reinterpret_cast<const float4*>(an + (w * 4 + g) * RP + j);
+            o.x += pa.x * f; o.y += pa.y * f; o.z += pa.z * f; o.w += pa.w * f;
+            nt.x += pn.x; nt.y += pn.y; nt.z += pn.z; nt.w += pn.w;
         }
         float* rec = a.part + (rec_base + g) * REC;
-        rec[4 + j] = o;
-        rec[4 + D + j] = nt;
-        if (j == 0) {
-            rec[0] = M;
-            rec[1] = l;
-            rec[2] = dt;
-            rec[3] = 0.f;
-        }
+        *reinterpret_cast<float4*>(rec + 4 + j) = o;
+        *reinterpret_cast<float4*>(rec + 4 + D + j) = nt;
+        if (j == 0) *reinterpret_cast<float4*>(rec) = make_float4(M, l, dt, 0.f);
     }
 }
 
@@ -778,8 +852,8 @@ static cudaError_t launch_mma_t(const CacheView& c, const CUtensorMap& tk, const
 
 // The merge area reuses the stage ring; it must fit.
 constexpr int kMaxSplit = 512;
-static_assert(2 * MmaCfg<128, 1, 2>::STAGE_BYTES >= (2 * 4 * 4 * 128 + 64) * 4, "merge area");
-static_assert(4 * MmaCfg<64, 1, 4>::STAGE_BYTES >= (2 * 4 * 4 * 64 + 64) * 4, "merge area");
+static_assert(2 * MmaCfg<128, 1, 2>::STAGE_BYTES >= (2 * 4 * 4 * 132 + 16 + 48) * 4, "merge area");
+static_assert(4 * MmaCfg<64, 1, 4>::STAGE_BYTES >= (2 * 4 * 4 * 68 + 16 + 48) * 4, "merge area");
 
 size_t mma_smem_for(int d, int bs, int max_per) {
     if (d == 128) return bs == 64 ? mma_smem_bytes<128, 1, 2>(max_per) : mma_smem_bytes<128, 2, 2>(max_per);
