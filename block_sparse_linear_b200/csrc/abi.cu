@@ -100,7 +100,8 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     const int G = p->num_q_heads / p->num_kv_heads;
     const int groups = batch * p->num_kv_heads;
     L.kcap = p->top_k + p->n_sink + p->n_local;
-    L.nw = (mbp + 31) / 32;
+    // a head's bitset row starts on 16 bytes (the decode kernel loads it as int4)
+    L.nw = ((mbp + 31) / 32 + 3) & ~3;
     L.rec = rec_floats(p->head_dim);
     const int umax = (int)std::min<int64_t>(mbp, (int64_t)G * L.kcap);
     // one wave: as many splits per group as fit the resident CTA slots, at least 2 blocks each
@@ -249,6 +250,11 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     if (st != SPLA_OK) return st;
     if ((st = check_cache(cache)) != SPLA_OK) return st;
     if (!q || !out) return SPLA_ERR_INVALID_ARG;
+    // the kernels move these by bulk copies, TMA boxes and 16-byte vector loads
+    auto misaligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) != 0; };
+    if (misaligned(q) || misaligned(cache->S) || misaligned(cache->z) || misaligned(cache->m) ||
+        misaligned(cache->blk_stats) || misaligned(cache->k_pool) || misaligned(cache->v_pool))
+        return SPLA_ERR_INVALID_ARG;
     const DecodeLayout L = layout_of(params, cache->batch, cache->max_blocks_per_seq);
     if (!workspace || workspace_bytes < L.total) return SPLA_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return SPLA_ERR_WORKSPACE;

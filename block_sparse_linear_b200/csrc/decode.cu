@@ -65,6 +65,81 @@ __device__ __noinline__ void stage_query(const void* q, const float* aw_ws, cons
     }
 }
 
+// Tensor-core path, before the dependency wait, one round of 16-byte loads (all
+// issued before any shared-memory store): the group's G query rows as raw bf16
+// (qraw[g][d]), the phi weights aw[i][4] = exp(q_g,i + m_i - c_g) the scoring
+// kernel used for the global readout (the kept blocks' term uses the very same
+// weights), m_i * log2e (ml[d]) and, with trow non-null, the sequence's
+// block-table row (its entry j at trow[j]). (Out of line, scalar arguments: the
+// prologue does not add to the register pressure of the streaming loop.)
+__device__ __noinline__ void stage_query_vec(const __nv_bfloat16* q, const float* aw_ws,
+                                             const float* m, const int32_t* table, int mbp,
+                                             int hq, int hkv, int G, int d, int b, int h,
+                                             uint32_t* qraw, float* aw, float* ml,
+                                             int32_t* trow_area, int32_t** trow, int tid,
+                                             int nthr) {
+    const int gi = b * hkv + h;
+    const int4* srcq = reinterpret_cast<const int4*>(q + ((int64_t)b * hq + h * G) * d);
+    const int4* srca = reinterpret_cast<const int4*>(aw_ws + (int64_t)gi * d * 4);
+    const int4* srcm = reinterpret_cast<const int4*>(m + (int64_t)gi * d);
+    const int nq = G * d / 8, na = d, nm = d / 4;            // int4 counts
+    // the table row: from the 16-byte boundary at or before its start; whole int4
+    // chunks that end inside the row, then the last few entries one by one
+    const int32_t* row = table + (int64_t)b * mbp;
+    const int off = trow_area ? (int)((reinterpret_cast<uintptr_t>(row) & 15) >> 2) : 0;
+    const int4* srct = reinterpret_cast<const int4*>(row - off);
+    const int nt = trow_area ? (off + mbp) / 4 : 0;
+    const int total = nq + na + nm + nt;
+    constexpr int kBatch = 8;
+    for (int e0 = tid; e0 < total; e0 += kBatch * nthr) {
+        int4 v[kBatch];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const int e = e0 + k * nthr;
+            if (e < nq) v[k] = __ldg(srcq + e);
+            else if (e < nq + na) v[k] = __ldcg(srca + (e - nq));
+            else if (e < nq + na + nm) v[k] = __ldcg(srcm + (e - nq - na));
+            else if (e < total) v[k] = __ldcg(srct + (e - nq - na - nm));
+        }
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const int e = e0 + k * nthr;
+            if (e < nq) reinterpret_cast<int4*>(qraw)[e] = v[k];
+            else if (e < nq + na) reinterpret_cast<int4*>(aw)[e - nq] = v[k];
+            else if (e < nq + na + nm) {
+                const int4 x = v[k];
+                float4 f = make_float4(__int_as_float(x.x) * SPLA_LOG2E, __int_as_float(x.y) * SPLA_LOG2E,
+                                       __int_as_float(x.z) * SPLA_LOG2E, __int_as_float(x.w) * SPLA_LOG2E);
+                reinterpret_cast<float4*>(ml)[e - nq - na] = f;
+            } else if (e < total) {
+                reinterpret_cast<int4*>(trow_area)[e - nq - na - nm] = v[k];
+            }
+        }
+    }
+    if (trow_area) {
+        for (int j = nt * 4 + tid; j < off + mbp; j += nthr) trow_area[j] = __ldcg(row - off + j);
+        *trow = trow_area + off;
+    }
+}
+
+// After the wait, one round of 16-byte loads: the G heads' selection bitset rows
+// (stride nw, a multiple of 4 words) into wbits[G][nw].
+__device__ __noinline__ void stage_bits_vec(const uint32_t* bits, int nw, int hq, int G, int b,
+                                            int h, uint32_t* wbits, int tid, int nthr) {
+    const int4* src = reinterpret_cast<const int4*>(bits + ((int64_t)b * hq + h * G) * nw);
+    const int n4 = G * nw / 4;
+    constexpr int kBatch = 4;
+    for (int e0 = tid; e0 < n4; e0 += kBatch * nthr) {
+        int4 v[kBatch];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k)
+            if (e0 + k * nthr < n4) v[k] = __ldcg(src + e0 + k * nthr);
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k)
+            if (e0 + k * nthr < n4) reinterpret_cast<int4*>(wbits)[e0 + k * nthr] = v[k];
+    }
+}
+
 // After the wait, one round of loads: the G heads' selection bitset words of
 // this group into wbits ([G][nwu], shared memory).
 __device__ __forceinline__ void stage_bits(const uint32_t* bits, int nw, int hq, int G, int b,
@@ -160,13 +235,14 @@ __device__ __noinline__ int union_share(const int32_t* trow, int num_phys, int G
 // physical blocks. No CTA barrier inside, and no lane walks more than one word
 // per sweep step.
 __device__ __forceinline__ int union_share_warp(const int32_t* trow, int num_phys, int G,
-                                                const uint32_t* wbits, int nwu, int nb, int split,
-                                                int nsplit, int max_per, int32_t* blk,
+                                                const uint32_t* wbits, int ws, int nwu, int nb,
+                                                int split, int nsplit, int max_per, int32_t* blk,
                                                 int32_t* phys, uint32_t* hm, int32_t* status,
                                                 int lane) {
+    // wbits: [G][ws] words, the first nwu of each row in use
     auto word = [&](int w) -> uint32_t {
         uint32_t u = 0u;
-        for (int g = 0; g < G; ++g) u |= wbits[g * nwu + w];
+        for (int g = 0; g < G; ++g) u |= wbits[g * ws + w];
         if (w == nwu - 1 && (nb & 31)) u &= (1u << (nb & 31)) - 1u;
         return u;
     };
@@ -199,7 +275,7 @@ __device__ __forceinline__ int union_share_warp(const int32_t* trow, int num_phy
                 if (r >= u0 && r < u1 && r - u0 < max_per) {
                     const int e = r - u0, j = (w << 5) + bit;
                     uint32_t mask = 0u;
-                    for (int g = 0; g < G; ++g) mask |= ((wbits[g * nwu + w] >> bit) & 1u) << g;
+                    for (int g = 0; g < G; ++g) mask |= ((wbits[g * ws + w] >> bit) & 1u) << g;
                     int32_t p = trow[j];
                     if (p < 0 || p >= num_phys) {
                         // read nothing from it: no head attends to it
@@ -384,13 +460,20 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         s_abort = 0;
     }
     const int nwu = (nb + 31) >> 5;
+    // the group's bitset rows [G][nw] and the table row borrow the stage buffers
+    // (no TMA in flight yet); the table row goes there whole when it fits and the
+    // table is 16-byte aligned, else its entries are read from global memory
     uint32_t* wbits = reinterpret_cast<uint32_t*>(stages);
-    const int trow_off = ((G + 1) * nwu + 3) & ~3;
-    int32_t* trow = reinterpret_cast<int32_t*>(wbits + trow_off);
-    const bool trow_smem = (size_t)(trow_off + c.mbp) * 4 <= (size_t)STAGES * Cfg::STAGE_BYTES;
-    stage_query(a.q, a.aw, c.m, c.table, c.mbp, c.hq, c.hkv, G, D, 1, b, h, qs, ml, aw,
-                (nb > 0 && trow_smem) ? trow : nullptr, tid, blockDim.x);
+    int32_t* trow_area = reinterpret_cast<int32_t*>(wbits + G4 * a.nw);
+    const bool trow_smem = ((reinterpret_cast<uintptr_t>(c.table) & 15) == 0) &&
+                           (size_t)(G4 * a.nw + c.mbp + 4) * 4 <= (size_t)STAGES * Cfg::STAGE_BYTES;
+    __shared__ int32_t* s_trow;
+    uint32_t* qraw = reinterpret_cast<uint32_t*>(qs);       // [G][D] bf16 pairs
+    stage_query_vec(static_cast<const __nv_bfloat16*>(a.q), a.aw, c.m, c.table, c.mbp, c.hq, c.hkv,
+                    G, D, b, h, qraw, aw, ml, (nb > 0 && trow_smem) ? trow_area : nullptr,
+                    &s_trow, tid, blockDim.x);
     __syncthreads();
+    const int32_t* trow = (nb > 0 && trow_smem) ? s_trow : c.table + (int64_t)b * c.mbp;
     // consumers' B fragments, still before the wait: column n = lane/4; rows
     // k = 2*(lane%4) (+1, +8, +9) of each 16-dim step
     uint32_t qf[D / 16][2], wf[D / 16][2];
@@ -402,11 +485,11 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int i = kb + 8 * half;
-                qf[kk][half] = (n < G) ? pack_bf16(qs[n * D + i], qs[n * D + i + 1]) : 0u;
+                qf[kk][half] = (n < G) ? qraw[(n * D + i) >> 1] : 0u;
                 uint32_t wv = 0u;
                 const int g = n & 3;
                 if (g < G) {
-                    const float x0 = aw[g * D + i], x1 = aw[g * D + i + 1];
+                    const float x0 = aw[i * 4 + g], x1 = aw[(i + 1) * 4 + g];
                     const uint32_t hi = pack_bf16(x0, x1);
                     wv = (n < 4) ? hi : pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
                 }
@@ -418,12 +501,11 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
     // the group's selections (one round of loads by every thread), then the producer
     // warp alone builds this CTA's share of their union
     if (nb > 0) {
-        stage_bits(a.bits, a.nw, c.hq, G, b, h, nwu, wbits, tid, blockDim.x);
+        stage_bits_vec(a.bits, a.nw, c.hq, G, b, h, wbits, tid, blockDim.x);
         __syncthreads();
         if (warp == NCW) {
-            const int n = union_share_warp(trow_smem ? trow : c.table + (int64_t)b * c.mbp,
-                                           c.num_phys, G, wbits, nwu, nb, split, nsplit,
-                                           a.max_per, blk, phys, hm, a.status, lane);
+            const int n = union_share_warp(trow, c.num_phys, G, wbits, a.nw, nwu, nb, split,
+                                           nsplit, a.max_per, blk, phys, hm, a.status, lane);
             if (lane == 0) s_n[0] = n;
         }
     } else if (tid == 0) {

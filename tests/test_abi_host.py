@@ -138,3 +138,16 @@ def test_static_workspace_entry_rejects_oversize_shapes_on_the_host(lib):
     with pytest.raises(_lib.SplaError) as e:
         _lib.spla_decode_static_workspace(p, c, FAKE, 0, FAKE, 0, 0, 0, 0)
     assert e.value.status == _lib.SPLA_ERR_CAPACITY
+
+
+def test_decode_rejects_misaligned_buffers(lib):
+    """q and the cache buffers the kernels move with bulk copies must be 16-byte aligned."""
+    B = ctypes.byref
+    p = _params()
+    need = _lib.spla_decode_workspace_size(p, 4, 2064)
+    assert lib.spla_decode(B(p), B(_cache()), FAKE + 2, None, FAKE, None, None, None, FAKE, need,
+                           None, None) == _lib.SPLA_ERR_INVALID_ARG
+    for field in ("S", "z", "m", "blk_stats", "k_pool", "v_pool"):
+        c = _cache(**{field: FAKE + 4})
+        assert lib.spla_decode(B(p), B(c), FAKE, None, FAKE, None, None, None, FAKE, need, None,
+                               None) == _lib.SPLA_ERR_INVALID_ARG, field
