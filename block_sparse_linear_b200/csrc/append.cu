@@ -67,7 +67,29 @@ __device__ void append_block(const CacheView& c, const T* k_new, const T* v_new,
     // statistics over all tokens now in the block: stage the keys in shared
     // memory with coalesced loads, then two passes per dimension in fp64
     const int nj = t_end - (int)blk_lo;
-    for (int e = threadIdx.x; e < nj * d; e += blockDim.x) ktile[e] = to_f(kp[e]);
+    {
+        // 16-byte loads, a batch of them in flight before any store (d is a multiple
+        // of 64, so a block's nj*d keys split into whole vectors)
+        constexpr int EPV = 16 / sizeof(T);
+        const int nvec = nj * d / EPV;
+        const int4* src = reinterpret_cast<const int4*>(kp);
+        constexpr int kBatch = 4;
+        for (int v0 = threadIdx.x; v0 < nvec; v0 += kBatch * blockDim.x) {
+            int4 x[kBatch];
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k)
+                if (v0 + k * (int)blockDim.x < nvec) x[k] = src[v0 + k * blockDim.x];
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+                const int v = v0 + k * blockDim.x;
+                if (v < nvec) {
+                    const T* e = reinterpret_cast<const T*>(&x[k]);
+#pragma unroll
+                    for (int u = 0; u < EPV; ++u) ktile[v * EPV + u] = to_f(e[u]);
+                }
+            }
+        }
+    }
     __syncthreads();
     float* st = c.stats + (((int64_t)b * c.hkv + h) * c.mbp + lb) * 2 * d;
     const int parts = blockDim.x / d;                // threads per dimension (2 at d=128, 4 at 64)

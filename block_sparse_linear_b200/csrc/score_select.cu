@@ -474,10 +474,24 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
     if (tid == 0) { s_min = 0xffffffffu; s_max = 0u; }
     __syncthreads();
     uint32_t lmin = 0xffffffffu, lmax = 0u;
-    for (int j = tid; j < nb; j += kSelThreads) {
-        const uint32_t k = forced(j) ? 0u : ordered_key(sc[j]);
-        keys[j] = k;
-        if (k) { lmin = min(lmin, k); lmax = max(lmax, k); }
+    // a batch of score loads in flight before any key is formed
+    constexpr int kKeyBatch = 8;
+    for (int j0 = tid; j0 < nb; j0 += kKeyBatch * kSelThreads) {
+        float x[kKeyBatch];
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+            const int j = j0 + u * kSelThreads;
+            x[u] = (j < nb) ? __ldcg(sc + j) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+            const int j = j0 + u * kSelThreads;
+            if (j < nb) {
+                const uint32_t k = forced(j) ? 0u : ordered_key(x[u]);
+                keys[j] = k;
+                if (k) { lmin = min(lmin, k); lmax = max(lmax, k); }
+            }
+        }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
