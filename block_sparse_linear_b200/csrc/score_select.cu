@@ -6,8 +6,8 @@
 //
 // score_kernel  persistent grid (2 CTAs of 4 warps per SM), every warp its
 //               own TMA pipeline over equal 32 KiB items: 32-block tiles of
-//               the statistics (lane l scores block l of the tile for all G
-//               heads with fp64 dot products, no lane reduction) and row
+//               the statistics (fp64 tensor-core dot products with the means,
+//               fp32 sums of the non-negative variance terms) and row
 //               ranges of the global state S for the linear-attention readout
 //               N, D that the combine step subtracts from.
 // select_kernel grid (batch*Hq), 512 threads. Exact top-k by key-space
@@ -21,39 +21,43 @@
 namespace spla {
 
 // ------------------------------------------------------------------ scoring
-// One launch works through a list of equal-sized items, taken by the warps of a
-// persistent grid (warp w of NW takes items w, w + NW, ...):
+// One launch works through a list of equal-sized items, taken by the warp pairs
+// of a persistent grid (pair p of NP takes items p, p + NP, ...):
 //   items [0, groups*RP)       global readout of one (sequence, KV head) group,
 //                              part p of RP row ranges of S (RP = 2 at d = 128);
 //   items groups*RP + gi*ntile + t
 //                              scores of blocks 32t .. 32t+31 of group gi.
-// Each warp is its own pipeline: lane 0 keeps kScoreRing stages of 8 KiB in
-// flight on per-warp mbarriers, the whole warp consumes them in order.
+// Each pair is its own pipeline: lane 0 of its first warp keeps kScoreRing
+// stages of 8 KiB in flight on the pair's mbarriers; both warps consume every
+// stage (each its half of the blocks, or of the readout columns) and meet on
+// the pair's named barrier before the stage is refilled. Two warps per stage
+// keep the dependent fp64 chains of a stage short.
 //
 // Score tile: the statistics are a 2-D fp32 tensor [groups*mbp rows][2d] (mean,
 // then variance, logical block order); one stage is two 32 x 32 boxes (mean and
 // variance of 32 dimensions of 32 blocks) with 128-byte swizzle. The dot
 // products run on the fp64 tensor cores (mma m8n8k4 f64): A = 8 blocks x 4
 // dimensions of statistics, B = 4 dimensions x 8 columns, the columns being
-// q'_g (g < 4) and q'_g^2 (g >= 4), q' = q * softmax_scale. B stays in
-// registers for the whole group (D/4 fp64 per lane); mean tiles accumulate
-// into one C, variance tiles into another, and the useful halves (mean x q',
-// variance x q'^2) are paired across lanes at the end. Rows of an A fragment
-// are blocks r/2 + 4(r%2) of an 8-block group, which keeps every quarter
-// warp's 16-byte reads on distinct bank groups under the swizzle.
+// q'_g (g < 4) and q'_g^2 (g >= 4), q' = q * softmax_scale (columns past G
+// are 0). Mean tiles accumulate into one C, variance tiles into another, and
+// the useful halves (mean x q', variance x q'^2) are paired across lanes at
+// the end. Rows of an A fragment are blocks r/2 + 4(r%2) of an 8-block group,
+// which keeps every quarter warp's 16-byte reads on distinct bank groups under
+// the swizzle; warp h of a pair takes the 8-block groups 2h and 2h + 1.
 //
 // Readout part: N[g][j] += sum_i a_g,i S[i][j], D[g] += sum_i a_g,i z_i over
 // its rows i, with a_g,i = exp(q_g,i + m_i - c_g), c_g = max over all i of
 // q_g,i + m_i (the same in every part, so the parts add). S rows arrive by 1-D
-// bulk copies; lane l owns columns l*d/32 ...
+// bulk copies; warp h of the pair owns columns [h d/2, (h+1) d/2).
 //
 // Nothing on the streaming path is read with ordinary loads: while the memory
 // system is saturated with bulk traffic those take microseconds to return. An
 // item's query rows (and m, z for a readout) arrive by bulk copy on a second
-// per-warp barrier, issued with the item's first stage; sequence lengths are
+// per-pair barrier, issued with the item's first stage; sequence lengths are
 // read into shared memory once at the start.
-constexpr int kScoreWarps = 4;          // warps per CTA
-constexpr int kScoreRing = 2;           // stages in flight per warp
+constexpr int kScorePairs = 4;          // warp pairs per CTA
+constexpr int kScoreWarps = 2 * kScorePairs;
+constexpr int kScoreRing = 2;           // stages in flight per pair
 constexpr int kScoreStage = 8192;       // bytes per stage
 constexpr int kScoreCtasPerSm = 2;
 constexpr int kTile = 32;               // blocks per score item
@@ -71,10 +75,10 @@ struct ScoreShape {
     static constexpr int kAuxPad = 1024 * ((kAux + 1023) / 1024);
     // two input buffers: item k uses buffer k % 2, so the next item's copy never
     // lands in rows the current item still reads
-    static constexpr int kWarpBytes = kScoreRing * kScoreStage + kATab + 2 * kAuxPad;
-    static constexpr int kSmem = kScoreWarps * kWarpBytes + 1024;           // + alignment
+    static constexpr int kPairBytes = kScoreRing * kScoreStage + kATab + 2 * kAuxPad;
+    static constexpr int kSmem = kScorePairs * kPairBytes + 1024;           // + alignment
     static_assert(kReadoutParts >= 1 && kReadoutParts * kTileStages * kRowsPerStage == D, "parts");
-    static_assert(kWarpBytes % 1024 == 0, "ring alignment for the 128B swizzle");
+    static_assert(kPairBytes % 1024 == 0, "ring alignment for the 128B swizzle");
 };
 
 // D(8x8, f64) += A(8x4, row) * B(4x8, col); per lane a = A[lane/4][lane%4],
@@ -109,29 +113,35 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
              float* __restrict__ gread, float* __restrict__ aw_out, int ntile, int32_t* status) {
     using S = ScoreShape<D>;
     constexpr int RP = S::kReadoutParts, TS = S::kTileStages, RPS = S::kRowsPerStage;
-    constexpr int CPL = D / 32;                    // readout columns per lane
+    constexpr int CPL = D / 32;                    // rows per lane in the readout weights
+    constexpr int HC = D / 2;                      // readout columns per warp
+    constexpr int CPH = HC / 32;                   // readout columns per lane
     extern __shared__ unsigned char smem_raw[];
-    __shared__ uint64_t full[kScoreWarps][kScoreRing];
-    __shared__ uint64_t qfull[kScoreWarps][2];
+    __shared__ uint64_t full[kScorePairs][kScoreRing];
+    __shared__ uint64_t qfull[kScorePairs][2];
     __shared__ int s_nb[kScoreNbSmem], s_len[kScoreNbSmem];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    unsigned char* base = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* ring = base + warp * S::kWarpBytes;
+    const int pair = warp >> 1, half = warp & 1;
+    // 1024-byte alignment by shared-pointer arithmetic (keeps the accesses ld.shared)
+    unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    unsigned char* ring = base + pair * S::kPairBytes;
     float* at = reinterpret_cast<float*>(ring + kScoreRing * kScoreStage);    // readout [D][4]
     unsigned char* aux0 = ring + kScoreRing * kScoreStage + S::kATab;          // q rows, m, z (x2)
-    uint64_t* bar = full[warp];
-    uint64_t* qbar = qfull[warp];
-    const int G = c.group;
-    const int groups = c.batch * c.hkv;
+    uint64_t* bar = full[pair];
+    uint64_t* qbar = qfull[pair];
+    const int G = c.group, hkv = c.hkv, mbp = c.mbp, bs = c.bs;
+    const int groups = c.batch * hkv;
     const int nread = groups * RP;
     const int nitems = nread + groups * ntile;
-    const int NW = gridDim.x * kScoreWarps;
-    const int wg = blockIdx.x * kScoreWarps + warp;
+    const int NP = gridDim.x * kScorePairs;
+    const int wp = blockIdx.x * kScorePairs + pair;
+    const bool leader = half == 0 && lane == 0;     // the pair's producer thread
+    const uint32_t pair_bar = 1u + (uint32_t)pair;  // named barrier of the pair (0 is __syncthreads)
+    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" :: "r"(pair_bar) : "memory"); };
 
     pdl_trigger();
     if (threadIdx.x == 0) prefetch_tmap(&tstats);
-    if (lane == 0) {
+    if (leader) {
         for (int s = 0; s < kScoreRing; ++s) mbar_init(&bar[s], 1);
         mbar_init(&qbar[0], 1);
         mbar_init(&qbar[1], 1);
@@ -140,30 +150,30 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
     pdl_wait();          // statistics, state and lengths come from the append kernels
     for (int b = threadIdx.x; b < min(c.batch, kScoreNbSmem); b += blockDim.x) {
         const int32_t L = c.lens[b];
-        if (blockIdx.x == 0 && (L < 0 || L > c.mbp * c.bs)) set_status(status, SPLA_DEV_CAPACITY);
-        s_len[b] = max(0, min(L, c.mbp * c.bs));
-        s_nb[b] = (s_len[b] + c.bs - 1) / c.bs;
+        if (blockIdx.x == 0 && (L < 0 || L > mbp * bs)) set_status(status, SPLA_DEV_CAPACITY);
+        s_len[b] = max(0, min(L, mbp * bs));
+        s_nb[b] = (s_len[b] + bs - 1) / bs;
     }
     __syncthreads();
     auto len_of = [&](int b) {
-        return b < kScoreNbSmem ? s_len[b] : max(0, min(c.lens[b], c.mbp * c.bs));
+        return b < kScoreNbSmem ? s_len[b] : max(0, min(c.lens[b], mbp * bs));
     };
     auto nb_of = [&](int b) {
         if (b < kScoreNbSmem) return s_nb[b];
-        return (len_of(b) + c.bs - 1) / c.bs;
+        return (len_of(b) + bs - 1) / bs;
     };
-    // next non-empty item at or after i in this warp's sequence
+    // next non-empty item at or after i in this pair's sequence
     auto next_item = [&](int i) {
-        for (; i < nitems; i += NW) {
+        for (; i < nitems; i += NP) {
             if (i < nread) return i;
             const int r = i - nread, gi = r / ntile, t = r % ntile;
-            if (t * kTile < nb_of(gi / c.hkv)) return i;
+            if (t * kTile < nb_of(gi / hkv)) return i;
         }
         return nitems;
     };
 
-    // ---- producer state (lane 0): item, stage within it, stages issued
-    int pi = next_item(wg), ps = 0, fi = 0, pk = 0;     // pk: items issued
+    // ---- producer state (the leader): item, stage within it, stages issued
+    int pi = next_item(wp), ps = 0, fi = 0, pk = 0;     // pk: items issued
     auto issue = [&]() {
         if (pi >= nitems) return;
         const int slot = fi % kScoreRing;
@@ -171,7 +181,7 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
         if (ps == 0) {
             // the item's query rows (and m, z for a readout) on the item barrier
             const int gi = pi < nread ? pi / RP : (pi - nread) / ntile;
-            const int b = gi / c.hkv, h = gi % c.hkv;
+            const int b = gi / hkv, h = gi % hkv;
             const uint32_t qb = (uint32_t)(G * D * sizeof(T));
             unsigned char* ax = aux0 + (pk & 1) * S::kAuxPad;
             uint64_t* qb_bar = &qbar[pk & 1];
@@ -190,32 +200,31 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
             bulk_load(dst, src, kScoreStage, &bar[slot]);
         } else {
             const int r = pi - nread, gi = r / ntile, t = r % ntile;
-            const int y = gi * c.mbp + t * kTile;
+            const int y = gi * mbp + t * kTile;
             tma_load_2d(dst, &tstats, &bar[slot], ps * 32, y);
             tma_load_2d(dst + kScoreStage / 2, &tstats, &bar[slot], D + ps * 32, y);
         }
         ++fi;
         if (++ps == TS) {
             ps = 0;
-            pi = next_item(pi + NW);
+            pi = next_item(pi + NP);
         }
     };
-    if (lane == 0)
+    if (leader)
         for (int s = 0; s < kScoreRing; ++s) issue();
 
     int f = 0;                 // stages consumed
     int nq = 0;                // items started: buffer nq % 2, its phase (nq / 2) % 2
-    // after a failed wait lane 0 waits (bounded) for every copy it has in flight
+    // after a failed wait the leader waits (bounded) for every copy it has in flight
     auto drain = [&](int q_from) {
         set_status(status, SPLA_DEV_TIMEOUT);
         for (int k = f; k < fi; ++k) mbar_wait_bounded(&bar[k % kScoreRing], (k / kScoreRing) & 1);
         for (int k = q_from; k < pk; ++k) mbar_wait_bounded(&qbar[k & 1], (k >> 1) & 1);
     };
-    // every lane agrees on the outcome of a wait
+    // every lane of the warp agrees on the outcome of a wait; a warp that gives up
+    // returns, and its partner's next wait on a copy that never comes gives up too
     auto wait_stage = [&](int slot) -> bool {
-        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar[slot], (f / kScoreRing) & 1));
-        if (!ok && lane == 0) drain(nq);
-        return ok;
+        return __all_sync(0xffffffffu, mbar_wait_bounded(&bar[slot], (f / kScoreRing) & 1));
     };
     const T* qs = nullptr;
     const float* ms = nullptr;
@@ -226,19 +235,42 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
         qs = reinterpret_cast<const T*>(ax);
         ms = reinterpret_cast<const float*>(ax + S::kQBytes);
         zs_ = ms + D;
-        if (!ok && lane == 0) drain(nq);
         ++nq;
         return ok;
     };
     const int kq = lane & 3, rq = lane >> 2;
+    const int prow = (rq >> 1) + 4 * (rq & 1);          // block row of A row rq in a group of 8
+    // swizzled offsets of this lane's A fragments: [8-block group of this warp][k half]
+    uint32_t aoff[2][2];
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) aoff[mi][hf] = swz128(8 * (2 * half + mi) + prow, 4 * hf + kq);
+    // both warps of a pair take every wait's outcome together: a failed wait sets
+    // the pair's flag, and after the next pair barrier both leave
+    __shared__ int s_fail[kScorePairs];
+    if (leader) s_fail[pair] = 0;
+    pair_sync();
+    // q_from: the first item copy that may still be in flight
+    auto agree = [&](bool ok, int q_from) -> bool {
+        if (!ok && lane == 0) s_fail[pair] = 1;
+        pair_sync();
+        if (s_fail[pair]) {
+            if (leader) drain(q_from);
+            return false;
+        }
+        return true;
+    };
 
-    for (int i = next_item(wg); i < nitems; i = next_item(i + NW)) {
+    for (int i = next_item(wp); i < nitems; i = next_item(i + NP)) {
         if (i < nread) {
-            // ---------------- global readout, rows of part `part`
+            // ---------------- global readout, rows of part `part`, columns of this warp
             const int gi = i / RP, part = i % RP;
             float dsum[4];
-            if (!wait_item()) return;
-            __syncwarp();                  // the previous readout's reads of `at` are done
+            {
+                const bool okq = wait_item();     // advances nq
+                if (!agree(okq, nq - 1)) return;
+            }
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
                 dsum[g] = 0.f;
@@ -256,71 +288,79 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
                     for (int u = 0; u < CPL; ++u) {
                         const int r = lane + 32 * u;
                         const float a = (mx == -SPLA_INF) ? 0.f : expf(v[u] - mx);
-                        at[r * 4 + g] = a;
+                        // each warp writes its half of the rows; both read all of them
+                        if ((r >= HC) == (half == 1)) at[r * 4 + g] = a;
                         if (r / (D / RP) == part) zs = fmaf(a, zs_[r], zs);
                     }
                     dsum[g] = warp_sum(zs);
                 } else {
 #pragma unroll
-                    for (int u = 0; u < CPL; ++u) at[(lane + 32 * u) * 4 + g] = 0.f;
+                    for (int u = 0; u < CPL; ++u) {
+                        const int r = lane + 32 * u;
+                        if ((r >= HC) == (half == 1)) at[r * 4 + g] = 0.f;
+                    }
                 }
             }
-            __syncwarp();
+            pair_sync();                   // the whole weight table is written
             if (part == 0) {
                 // the decode kernels weight phi(k) with the same a_g,i
                 float4* awg = reinterpret_cast<float4*>(aw_out + (int64_t)gi * D * 4);
-                for (int r = lane; r < D; r += 32) awg[r] = *reinterpret_cast<const float4*>(at + r * 4);
+                for (int r = half * HC + lane; r < (half + 1) * HC; r += 32)
+                    awg[r] = *reinterpret_cast<const float4*>(at + r * 4);
             }
-            float acc[4][CPL];
+            float acc[4][CPH];
 #pragma unroll
             for (int g = 0; g < 4; ++g)
 #pragma unroll
-                for (int u = 0; u < CPL; ++u) acc[g][u] = 0.f;
+                for (int u = 0; u < CPH; ++u) acc[g][u] = 0.f;
 #pragma unroll 1
             for (int s = 0; s < TS; ++s, ++f) {
                 const int slot = f % kScoreRing;
-                if (!wait_stage(slot)) return;
-                const float* sm = reinterpret_cast<const float*>(ring + slot * kScoreStage);
-                const int row0 = (part * TS + s) * RPS;
+                const bool ok = wait_stage(slot);
+                if (ok) {
+                    const float* sm = reinterpret_cast<const float*>(ring + slot * kScoreStage);
+                    const int row0 = (part * TS + s) * RPS;
 #pragma unroll 4
-                for (int r = 0; r < RPS; ++r) {
-                    const float4 a4 = *reinterpret_cast<const float4*>(at + (row0 + r) * 4);
-                    float sv[CPL];
-                    if constexpr (CPL == 4) {
-                        const float4 t4 = *reinterpret_cast<const float4*>(sm + r * D + lane * 4);
-                        sv[0] = t4.x; sv[1] = t4.y; sv[2] = t4.z; sv[3] = t4.w;
-                    } else {
-                        const float2 t2 = *reinterpret_cast<const float2*>(sm + r * D + lane * 2);
-                        sv[0] = t2.x; sv[1] = t2.y;
+                    for (int r = 0; r < RPS; ++r) {
+                        const float4 a4 = *reinterpret_cast<const float4*>(at + (row0 + r) * 4);
+                        float sv[CPH];
+                        if constexpr (CPH == 2) {
+                            const float2 t2 = *reinterpret_cast<const float2*>(sm + r * D + half * HC + lane * 2);
+                            sv[0] = t2.x; sv[1] = t2.y;
+                        } else {
+                            sv[0] = sm[r * D + half * HC + lane];
+                        }
+                        const float ag[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+#pragma unroll
+                            for (int u = 0; u < CPH; ++u) acc[g][u] = fmaf(ag[g], sv[u], acc[g][u]);
                     }
-                    const float ag[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                    for (int g = 0; g < 4; ++g)
-#pragma unroll
-                        for (int u = 0; u < CPL; ++u) acc[g][u] = fmaf(ag[g], sv[u], acc[g][u]);
                 }
-                __syncwarp();
-                if (lane == 0) issue();
+                if (!agree(ok, nq)) return;
+                if (leader) issue();
             }
             float* out = gread + ((int64_t)gi * RP + part) * G * (D + 4);
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
                 if (g < G) {
 #pragma unroll
-                    for (int u = 0; u < CPL; ++u) out[g * (D + 4) + lane * CPL + u] = acc[g][u];
-                    if (lane == 0) out[g * (D + 4) + D] = dsum[g];
+                    for (int u = 0; u < CPH; ++u) out[g * (D + 4) + half * HC + lane * CPH + u] = acc[g][u];
+                    if (half == 0 && lane == 0) out[g * (D + 4) + D] = dsum[g];
                 }
             }
             continue;
         }
-        // ---------------- score tile
+        // ---------------- score tile: this warp's 16 of the 32 blocks
         const int r = i - nread, gi = r / ntile, t = r % ntile;
-        const int b = gi / c.hkv, h = gi % c.hkv;
-        if (!wait_item()) return;
-        double cm[4][2], cs[4][2];
+        const int b = gi / hkv, h = gi % hkv;
+        {
+            const bool okq = wait_item();         // advances nq
+            if (!agree(okq, nq - 1)) return;
+        }
+        double cm[2][2], cs[2][2];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) cm[m][0] = cm[m][1] = cs[m][0] = cs[m][1] = 0.0;
-        const int prow = (rq >> 1) + 4 * (rq & 1);          // block row of A row rq in a group of 8
+        for (int mi = 0; mi < 2; ++mi) cm[mi][0] = cm[mi][1] = cs[mi][0] = cs[mi][1] = 0.0;
         const int head = rq & 3;
         const bool sq = rq >= 4;
         const T* qh = qs + head * D;
@@ -342,47 +382,48 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
                 }
             }
             const int slot = f % kScoreRing;
-            if (!wait_stage(slot)) return;
-            const unsigned char* st = ring + slot * kScoreStage;
+            const bool ok = wait_stage(slot);
+            if (ok) {
+                const unsigned char* st = ring + slot * kScoreStage;
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float mu[4][4], va[4][4];
+                for (int hf = 0; hf < 2; ++hf) {
+                    float mu[2][4], va[2][4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const uint32_t off = swz128(8 * m + prow, 4 * hf + kq);
-                    const float4 m4 = *reinterpret_cast<const float4*>(st + off);
-                    const float4 v4 = *reinterpret_cast<const float4*>(st + kScoreStage / 2 + off);
-                    mu[m][0] = m4.x; mu[m][1] = m4.y; mu[m][2] = m4.z; mu[m][3] = m4.w;
-                    va[m][0] = v4.x; va[m][1] = v4.y; va[m][2] = v4.z; va[m][3] = v4.w;
-                }
-                // eight independent accumulators per k-slice
+                    for (int mi = 0; mi < 2; ++mi) {
+                        const float4 m4 = *reinterpret_cast<const float4*>(st + aoff[mi][hf]);
+                        const float4 v4 = *reinterpret_cast<const float4*>(st + kScoreStage / 2 + aoff[mi][hf]);
+                        mu[mi][0] = m4.x; mu[mi][1] = m4.y; mu[mi][2] = m4.z; mu[mi][3] = m4.w;
+                        va[mi][0] = v4.x; va[mi][1] = v4.y; va[mi][2] = v4.z; va[mi][3] = v4.w;
+                    }
+                    // four independent accumulators per k-slice
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < 4; ++u) {
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        dmma_884(cm[m], (double)mu[m][u], bq[hf * 4 + u]);
-                        dmma_884(cs[m], (double)va[m][u], bq[hf * 4 + u]);
+                        for (int mi = 0; mi < 2; ++mi) {
+                            dmma_884(cm[mi], (double)mu[mi][u], bq[hf * 4 + u]);
+                            dmma_884(cs[mi], (double)va[mi][u], bq[hf * 4 + u]);
+                        }
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0) issue();
+            if (!agree(ok, nq)) return;
+            if (leader) issue();
         }
         // lanes kq < 2 hold mean x q' (columns 2kq, 2kq+1 = heads); their partners
         // kq + 2 hold variance x q'^2 for the same heads
         const int nbs = nb_of(b);
         const int32_t L = len_of(b);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const double mine0 = (kq < 2) ? cm[m][0] : cs[m][0];
-            const double mine1 = (kq < 2) ? cm[m][1] : cs[m][1];
+        for (int mi = 0; mi < 2; ++mi) {
+            const double mine0 = (kq < 2) ? cm[mi][0] : cs[mi][0];
+            const double mine1 = (kq < 2) ? cm[mi][1] : cs[mi][1];
             const double oth0 = __shfl_xor_sync(0xffffffffu, mine0, 2);
             const double oth1 = __shfl_xor_sync(0xffffffffu, mine1, 2);
-            const int j = t * kTile + 8 * m + prow;
+            const int j = t * kTile + 8 * (2 * half + mi) + prow;
             if (kq < 2 && j < nbs) {
-                const int nj = min(c.bs, L - j * c.bs);
+                const int nj = min(bs, L - j * bs);
                 // log n_j: a constant except for a sequence's last block
-                const double lg = (nj == c.bs) ? log_bs : c_log_n[nj];
+                const double lg = (nj == bs) ? log_bs : c_log_n[nj];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int g = 2 * kq + e;
@@ -393,7 +434,7 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
                             // while the argument stays below e^4 - 1
                             sc += (double)log1pf((float)(0.5 * (e ? oth1 : oth0)));
                         }
-                        scores[((int64_t)b * c.hq + h * G + g) * c.mbp + j] = (float)sc;
+                        scores[((int64_t)b * c.hq + h * G + g) * mbp + j] = (float)sc;
                     }
                 }
             }
@@ -403,8 +444,17 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
 
 // ------------------------------------------------------------------ selection
 constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kCandCap = 256;
+constexpr uint32_t kMark = 0xffffffffu;     // a selected key (only a NaN score maps here)
+constexpr int kWordsPerThread = SPLA_MAX_BLOCKS_PER_SEQ / 32 / kSelThreads;
+static_assert(kWordsPerThread * 32 * kSelThreads == SPLA_MAX_BLOCKS_PER_SEQ, "bitset words per thread");
+
+// The float a key was made from (the inverse of ordered_key).
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
 __device__ int block_excl_scan(int v, int* tmp, int* total) {
     // tmp: >= 33 ints of shared memory
@@ -434,6 +484,47 @@ __device__ int block_excl_scan(int v, int* tmp, int* total) {
     return before;
 }
 
+// Marks (kMark) the krem largest of the nc gathered candidates: one composite per
+// candidate, a larger key or an equal key at a lower block index comparing
+// greater. Starts and ends on a barrier-separated state.
+__device__ __forceinline__ void rank_candidates(uint32_t* keys, const uint32_t* cand_key,
+                                                const int* cand_idx, unsigned long long* cand_c,
+                                                int nc, int krem) {
+    const int tid = threadIdx.x;
+    const int ncp = (nc + 7) & ~7;
+    for (int i = tid; i < ncp; i += kSelThreads)
+        cand_c[i] = (i < nc) ? (((unsigned long long)cand_key[i] << 32) |
+                                (uint32_t)~(uint32_t)cand_idx[i])
+                             : 0ull;
+    __syncthreads();
+    for (int i = tid; i < nc; i += kSelThreads) {
+        const unsigned long long mine = cand_c[i];
+        int rank = 0;
+        // eight candidates per step, their loads in flight together
+        for (int o = 0; o < ncp; o += 8) {
+            const ulonglong2 x0 = *reinterpret_cast<const ulonglong2*>(cand_c + o);
+            const ulonglong2 x1 = *reinterpret_cast<const ulonglong2*>(cand_c + o + 2);
+            const ulonglong2 x2 = *reinterpret_cast<const ulonglong2*>(cand_c + o + 4);
+            const ulonglong2 x3 = *reinterpret_cast<const ulonglong2*>(cand_c + o + 6);
+            rank += (x0.x > mine) + (x0.y > mine) + (x1.x > mine) + (x1.y > mine) +
+                    (x2.x > mine) + (x2.y > mine) + (x3.x > mine) + (x3.y > mine);
+        }
+        if (rank < krem) keys[cand_idx[i]] = kMark;
+    }
+    __syncthreads();
+}
+
+// Selection of one head. Keys are the scores in a monotone uint32 order (forced
+// sink and local blocks get key 0 and are always kept).
+//   fast pass  2048 buckets linear in the score value over [min, max]: scores
+//              spread over many buckets, so the shared-memory counters see little
+//              contention; the bucket holding the k-th largest key is found by a
+//              suffix scan, every key above it is marked selected, and the bucket's
+//              keys (few) are ranked pairwise (ties -> lower block index).
+//   refinement (a non-finite score range, or more than kCandCap keys in that
+//              bucket) buckets linear in key space, narrowed pass by pass.
+// Every step that reads what another warp wrote is one barrier apart; no loop
+// carries a dependency through shared memory.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int top_k, int n_sink,
                                                              int n_local, const float* scores,
                                                              uint32_t* bits, int nw,
@@ -447,9 +538,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
     __shared__ int cand_idx[kCandCap];
     __shared__ __align__(16) unsigned long long cand_c[kCandCap];   // key << 32 | ~index
     __shared__ int tmp[40];
+    __shared__ uint32_t wmn[kSelWarps], wmx[kSelWarps];
     __shared__ unsigned long long s_lo, s_hi;
-    __shared__ int s_krem, s_cnt, s_done, s_mode, s_ncand, s_total;
-    __shared__ uint32_t s_min, s_max;
+    __shared__ int s_krem, s_cnt, s_done, s_mode, s_ncand, s_bstar;
 
     const int b = blockIdx.x / c.hq, hq = blockIdx.x % c.hq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -471,11 +562,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
     const int ncand = nb - nforced;
     const bool take_all = ncand <= top_k;
 
-    if (tid == 0) { s_min = 0xffffffffu; s_max = 0u; }
-    __syncthreads();
+    // ---- keys, their range, and cleared bucket counters
     uint32_t lmin = 0xffffffffu, lmax = 0u;
-    // a batch of score loads in flight before any key is formed
-    constexpr int kKeyBatch = 8;
+    constexpr int kKeyBatch = 8;                    // score loads in flight before any key is formed
     for (int j0 = tid; j0 < nb; j0 += kKeyBatch * kSelThreads) {
         float x[kKeyBatch];
 #pragma unroll
@@ -493,175 +582,238 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
             }
         }
     }
+    for (int i = tid; i < kBins; i += kSelThreads) hist[i] = 0;
+    if (tid == 0) { s_ncand = 0; s_bstar = -1; s_cnt = 0; s_krem = top_k; }
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
         lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
         lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
     }
-    if (lane == 0 && !take_all) {
-        atomicMin(&s_min, lmin);
-        atomicMax(&s_max, lmax);
-    }
+    if (lane == 0) { wmn[warp] = lmin; wmx[warp] = lmax; }
     __syncthreads();
 
+    unsigned long long thr = 0ull;                  // keys >= thr are selected
     if (!take_all) {
-        if (tid == 0) {
-            s_lo = s_min;
-            s_hi = (unsigned long long)s_max + 1ull;
-            s_krem = top_k;
-            s_done = 0;
-            s_mode = 0;
-        }
-        __syncthreads();
-        for (int pass = 0; pass < 8 && !s_done; ++pass) {
-            const unsigned long long lo = s_lo, hi = s_hi;
-            int shift = 0;
-            while (((hi - lo - 1ull) >> shift) >= (unsigned long long)kBins) ++shift;
-            const int nbins = (int)((hi - lo - 1ull) >> shift) + 1;
-            for (int i = tid; i < nbins; i += kSelThreads) hist[i] = 0;
-            __syncthreads();
+        uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+        for (int w = 0; w < kSelWarps; ++w) { kmin = min(kmin, wmn[w]); kmax = max(kmax, wmx[w]); }
+        const float fmin = key_value(kmin), fmax = key_value(kmax);
+        const float span = fmax - fmin;
+        // block-uniform: every thread computed the same range
+        const bool fast = isfinite(fmin) && isfinite(fmax) && span > 0.f && isfinite(span);
+        bool refine = !fast;
+        if (fast) {
+            const float scl = (float)kBins / span;
+            // monotone in the key: a larger key never lands in a lower bucket
+            auto fbin = [&](uint32_t k) {
+                return min(kBins - 1, max(0, (int)((key_value(k) - fmin) * scl)));
+            };
             for (int j = tid; j < nb; j += kSelThreads) {
-                const unsigned long long k = keys[j];
-                if (k >= lo && k < hi) atomicAdd(&hist[(int)((k - lo) >> shift)], 1);
+                const uint32_t k = keys[j];
+                if (k) atomicAdd(&hist[fbin(k)], 1);
             }
             __syncthreads();
             // suffix scan from the top bucket; thread t covers reversed buckets [4t, 4t+4)
             int local[4], lsum = 0;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int r = 4 * tid + u;
-                local[u] = (r < nbins) ? hist[nbins - 1 - r] : 0;
+                local[u] = hist[kBins - 1 - (4 * tid + u)];
                 lsum += local[u];
             }
             const int before = block_excl_scan(lsum, tmp, nullptr);
-            const int krem = s_krem;
-            if (before < krem && before + lsum >= krem) {
+            if (before < top_k && before + lsum >= top_k) {
                 int acc = before;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    if (acc < krem && acc + local[u] >= krem) {
-                        const int bstar = nbins - 1 - (4 * tid + u);
-                        const unsigned long long nlo = lo + ((unsigned long long)bstar << shift);
-                        unsigned long long nhi = lo + ((unsigned long long)(bstar + 1) << shift);
-                        if (nhi > hi) nhi = hi;
-                        s_lo = nlo;
-                        s_hi = nhi;
-                        s_krem = krem - acc;        // still to take from [nlo, nhi)
+                    if (acc < top_k && acc + local[u] >= top_k) {
+                        s_bstar = kBins - 1 - (4 * tid + u);
+                        s_krem = top_k - acc;        // still to take from the bucket
                         s_cnt = local[u];
                     }
                     acc += local[u];
                 }
             }
             __syncthreads();
-            if (tid == 0) {
-                if (s_cnt == s_krem) { s_mode = 1; s_done = 1; }            // the whole bucket
-                else if (s_cnt <= kCandCap) { s_mode = 2; s_done = 1; }     // rank candidates
-                else if (s_hi - s_lo == 1ull) { s_mode = 3; s_done = 1; }   // all equal: by index
-                else s_mode = 0;
-                s_ncand = 0;
+            const int bstar = s_bstar, krem = s_krem;
+            if (s_cnt <= kCandCap) {
+                // everything above the bucket is selected; the bucket's keys are candidates
+                for (int r = 0; r < rounds; ++r) {
+                    const int j = r * kSelThreads + tid;
+                    bool in = false;
+                    if (j < nb) {
+                        const uint32_t k = keys[j];
+                        if (k) {
+                            const int bb = fbin(k);
+                            if (bb > bstar) keys[j] = kMark;
+                            in = bb == bstar;
+                        }
+                    }
+                    const uint32_t m = __ballot_sync(0xffffffffu, in);
+                    int base = 0;
+                    if (lane == 0 && m) base = atomicAdd(&s_ncand, __popc(m));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (in) {
+                        const int p = base + __popc(m & ((1u << lane) - 1u));
+                        if (p < kCandCap) { cand_key[p] = keys[j]; cand_idx[p] = j; }
+                    }
+                }
+                __syncthreads();
+                rank_candidates(keys, cand_key, cand_idx, cand_c, min(s_ncand, kCandCap), krem);
+                thr = kMark;
+            } else {
+                // key range of the crowded bucket, then key-space refinement inside it
+                uint32_t bmin = 0xffffffffu, bmax = 0u;
+                for (int j = tid; j < nb; j += kSelThreads) {
+                    const uint32_t k = keys[j];
+                    if (k && fbin(k) == bstar) { bmin = min(bmin, k); bmax = max(bmax, k); }
+                }
+#pragma unroll
+                for (int o = 16; o; o >>= 1) {
+                    bmin = min(bmin, __shfl_xor_sync(0xffffffffu, bmin, o));
+                    bmax = max(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+                }
+                __syncthreads();                     // every thread has read wmn / wmx
+                if (lane == 0) { wmn[warp] = bmin; wmx[warp] = bmax; }
+                __syncthreads();
+                kmin = 0xffffffffu; kmax = 0u;
+#pragma unroll
+                for (int w = 0; w < kSelWarps; ++w) { kmin = min(kmin, wmn[w]); kmax = max(kmax, wmx[w]); }
+                if (tid == 0) { s_lo = kmin; s_hi = (unsigned long long)kmax + 1ull; }
+                refine = true;
             }
-            __syncthreads();
+        } else if (tid == 0) {
+            s_lo = kmin;
+            s_hi = (unsigned long long)kmax + 1ull;
+            s_krem = top_k;
         }
-        const unsigned long long lo = s_lo, hi = s_hi;
-        const int krem = s_krem;
-        if (s_mode == 1) {
-            // every key in [lo, hi) is selected: lift them above the final threshold
-            for (int j = tid; j < nb; j += kSelThreads)
-                if (keys[j] >= lo && keys[j] < hi) keys[j] = 0xffffffffu;
-        } else if (s_mode == 2) {
-            for (int r = 0; r < rounds; ++r) {
-                const int j = r * kSelThreads + tid;
-                const bool in = j < nb && keys[j] >= lo && keys[j] < hi;
-                const uint32_t m = __ballot_sync(0xffffffffu, in);
-                int base = 0;
-                if (lane == 0 && m) base = atomicAdd(&s_ncand, __popc(m));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                if (in) {
-                    const int p = base + __popc(m & ((1u << lane) - 1u));
-                    if (p < kCandCap) { cand_key[p] = keys[j]; cand_idx[p] = j; }
+        if (refine) {
+            if (tid == 0) { s_done = 0; s_mode = 0; }
+            __syncthreads();
+            for (int pass = 0; pass < 8 && !s_done; ++pass) {
+                const unsigned long long lo = s_lo, hi = s_hi;
+                // the smallest shift that maps [lo, hi) onto at most kBins buckets
+                const unsigned long long range = hi - lo - 1ull;
+                const int shift = max(0, 64 - __clzll((long long)range) - 11);
+                const int nbins = (int)(range >> shift) + 1;
+                for (int i = tid; i < nbins; i += kSelThreads) hist[i] = 0;
+                __syncthreads();
+                for (int j = tid; j < nb; j += kSelThreads) {
+                    const unsigned long long k = keys[j];
+                    if (k >= lo && k < hi) atomicAdd(&hist[(int)((k - lo) >> shift)], 1);
+                }
+                __syncthreads();
+                int local[4], lsum = 0;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = 4 * tid + u;
+                    local[u] = (r < nbins) ? hist[nbins - 1 - r] : 0;
+                    lsum += local[u];
+                }
+                const int before = block_excl_scan(lsum, tmp, nullptr);
+                const int krem = s_krem;
+                if (before < krem && before + lsum >= krem) {
+                    int acc = before;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (acc < krem && acc + local[u] >= krem) {
+                            const int bst = nbins - 1 - (4 * tid + u);
+                            const unsigned long long nlo = lo + ((unsigned long long)bst << shift);
+                            unsigned long long nhi = lo + ((unsigned long long)(bst + 1) << shift);
+                            if (nhi > hi) nhi = hi;
+                            s_lo = nlo;
+                            s_hi = nhi;
+                            s_krem = krem - acc;     // still to take from [nlo, nhi)
+                            s_cnt = local[u];
+                        }
+                        acc += local[u];
+                    }
+                }
+                __syncthreads();
+                if (tid == 0) {
+                    if (s_cnt == s_krem) { s_mode = 1; s_done = 1; }            // the whole bucket
+                    else if (s_cnt <= kCandCap) { s_mode = 2; s_done = 1; }     // rank candidates
+                    else if (s_hi - s_lo == 1ull) { s_mode = 3; s_done = 1; }   // all equal: by index
+                    else s_mode = 0;
+                    s_ncand = 0;
+                }
+                __syncthreads();
+            }
+            const unsigned long long lo = s_lo, hi = s_hi;
+            const int krem = s_krem;
+            if (s_mode == 1) {
+                // every key in [lo, hi) is selected
+                for (int j = tid; j < nb; j += kSelThreads)
+                    if (keys[j] >= lo && keys[j] < hi) keys[j] = kMark;
+            } else if (s_mode == 2) {
+                for (int r = 0; r < rounds; ++r) {
+                    const int j = r * kSelThreads + tid;
+                    const bool in = j < nb && keys[j] >= lo && keys[j] < hi;
+                    const uint32_t m = __ballot_sync(0xffffffffu, in);
+                    int base = 0;
+                    if (lane == 0 && m) base = atomicAdd(&s_ncand, __popc(m));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (in) {
+                        const int p = base + __popc(m & ((1u << lane) - 1u));
+                        if (p < kCandCap) { cand_key[p] = keys[j]; cand_idx[p] = j; }
+                    }
+                }
+                __syncthreads();
+                rank_candidates(keys, cand_key, cand_idx, cand_c, min(s_ncand, kCandCap), krem);
+            } else {
+                // equal keys: the krem lowest indices among keys == lo, in index order
+                int taken = 0;
+                for (int r = 0; r < rounds; ++r) {
+                    const int j = r * kSelThreads + tid;
+                    const bool eq = j < nb && keys[j] == lo;
+                    int tot;
+                    const int rank = taken + block_excl_scan(eq ? 1 : 0, tmp, &tot);
+                    if (eq && rank < krem) keys[j] = kMark;
+                    taken += tot;
                 }
             }
-            __syncthreads();
-            const int nc = min(s_ncand, kCandCap);
-            // one composite per candidate: a larger key, or an equal key at a lower
-            // block index, compares greater
-            const int ncp = (nc + 7) & ~7;
-            for (int i = tid; i < ncp; i += kSelThreads)
-                cand_c[i] = (i < nc) ? (((unsigned long long)cand_key[i] << 32) |
-                                        (uint32_t)~(uint32_t)cand_idx[i])
-                                     : 0ull;
-            __syncthreads();
-            for (int i = tid; i < nc; i += kSelThreads) {
-                const unsigned long long mine = cand_c[i];
-                int rank = 0;
-                // eight candidates per step, their loads in flight together
-                for (int o = 0; o < ncp; o += 8) {
-                    const ulonglong2 x0 = *reinterpret_cast<const ulonglong2*>(cand_c + o);
-                    const ulonglong2 x1 = *reinterpret_cast<const ulonglong2*>(cand_c + o + 2);
-                    const ulonglong2 x2 = *reinterpret_cast<const ulonglong2*>(cand_c + o + 4);
-                    const ulonglong2 x3 = *reinterpret_cast<const ulonglong2*>(cand_c + o + 6);
-                    rank += (x0.x > mine) + (x0.y > mine) + (x1.x > mine) + (x1.y > mine) +
-                            (x2.x > mine) + (x2.y > mine) + (x3.x > mine) + (x3.y > mine);
-                }
-                if (rank < krem) keys[cand_idx[i]] = 0xffffffffu;
-            }
-        } else {
-            // equal keys: the krem lowest indices among keys == lo, in index order
-            int taken = 0;
-            for (int r = 0; r < rounds; ++r) {
-                const int j = r * kSelThreads + tid;
-                const bool eq = j < nb && keys[j] == lo;
-                int tot;
-                const int rank = taken + block_excl_scan(eq ? 1 : 0, tmp, &tot);
-                if (eq && rank < krem) keys[j] = 0xffffffffu;
-                taken += tot;
-            }
+            thr = hi;
         }
         __syncthreads();
     }
 
-    // flags -> bitset words (one ballot per 32 consecutive blocks), then list positions
-    const unsigned long long thr = take_all ? 0ull : s_hi;
+    // ---- flags -> bitset words (one ballot per 32 consecutive blocks), then list positions
     uint32_t* hb = bits + ((int64_t)b * c.hq + hq) * nw;
     const int nwu = (nb + 31) >> 5;
     for (int r = 0; r < rounds; ++r) {
         const int j = r * kSelThreads + tid;
         const bool sel = j < nb && (take_all || forced(j) || (unsigned long long)keys[j] >= thr);
         const uint32_t word = __ballot_sync(0xffffffffu, sel);
-        const int wi = (r * kSelThreads + warp * 32) >> 5;
+        const int wi = r * kSelWarps + warp;
         if (lane == 0 && wi < nwu) {
             hb[wi] = word;
             wpre[wi] = __popc(word);
         }
     }
     __syncthreads();
-    if (warp == 0) {
-        // exclusive scan of the per-word counts, 32 consecutive words per lane
-        const int wpl = (nwu + 31) >> 5;
-        const int w0 = lane * wpl, w1 = min(nwu, w0 + wpl);
-        int cnt = 0;
-        for (int w = w0; w < w1; ++w) cnt += wpre[w];
-        int x = cnt;
+    // exclusive scan of the word counts: thread t owns words [t * W, t * W + W)
+    int total;
+    {
+        int cw[kWordsPerThread], v = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+        for (int u = 0; u < kWordsPerThread; ++u) {
+            const int w = tid * kWordsPerThread + u;
+            cw[u] = w < nwu ? wpre[w] : 0;
+            v += cw[u];
         }
-        int run = x - cnt;
-        for (int w = w0; w < w1; ++w) {
-            const int v = wpre[w];
-            wpre[w] = run;
-            run += v;
+        int run = block_excl_scan(v, tmp, &total);
+#pragma unroll
+        for (int u = 0; u < kWordsPerThread; ++u) {
+            const int w = tid * kWordsPerThread + u;
+            if (w < nwu) wpre[w] = run;
+            run += cw[u];
         }
-        if (lane == 31) s_total = x;
     }
     __syncthreads();
-    const int total = s_total;
     if (sel_idx) {
         int32_t* out = sel_idx + ((int64_t)b * c.hq + hq) * kcap;
         for (int r = 0; r < rounds; ++r) {
             const int j = r * kSelThreads + tid;
-            const int wi = (r * kSelThreads + warp * 32) >> 5;
+            const int wi = r * kSelWarps + warp;
             if (wi < nwu) {
                 const uint32_t word = hb[wi];
                 if ((word >> lane) & 1u) {
@@ -683,7 +835,7 @@ static cudaError_t launch_score_t(const CacheView& c, const CUtensorMap& tstats,
     const int groups = c.batch * c.hkv;
     const int ntile = (c.mbp + kTile - 1) / kTile;
     const int64_t nitems = (int64_t)groups * (S::kReadoutParts + ntile);
-    const int grid = (int)std::min<int64_t>((nitems + kScoreWarps - 1) / kScoreWarps,
+    const int grid = (int)std::min<int64_t>((nitems + kScorePairs - 1) / kScorePairs,
                                             (int64_t)kScoreCtasPerSm * kNumSms);
     cudaError_t e = cudaFuncSetAttribute(score_kernel<D, T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);

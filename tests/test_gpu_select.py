@@ -1,0 +1,121 @@
+"""Top-k selection edge cases on the GPU: exact ties and crowded score buckets.
+
+The caches are filled from hand-made fp32 keys: every block is one base
+pattern plus an offset along a fixed direction, so a block's score is an affine
+function of its offset and classes of blocks can share a score exactly. The
+selection rule (the top_k largest estimates, equal estimates taken in block
+order, sink and local blocks always kept) is checked directly, and every head
+is also compared with the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_linear_b200 import SplaDecodeCache
+from oracle import feed as ofeed
+from oracle import spla_oracle as so
+from workloads import feed_gpu, gen
+
+from . import parity
+
+pytestmark = pytest.mark.gpu
+
+CHUNK = 4096          # whole blocks per append, so every block's statistics come from one call
+
+
+def _workload(n_blocks):
+    return gen.scaled("cfg3", context_lens=(64 * n_blocks,), dtype="f32", top_k=32,
+                      n_sink=1, n_local=1, extra_tokens=0)
+
+
+def _direction(q, w):
+    """Unit vector per KV head along the sum of its query heads."""
+    u = q[0].reshape(w.num_kv_heads, w.num_q_heads // w.num_kv_heads, w.head_dim).sum(axis=1)
+    return u / np.linalg.norm(u, axis=1, keepdims=True)
+
+
+def _keys(w, t, q, seed):
+    """K, V [L][Hkv][d]: block j = base pattern + t[j] * u (per KV head)."""
+    rng = np.random.default_rng(seed)
+    bs, H, d = w.block_size, w.num_kv_heads, w.head_dim
+    base = rng.standard_normal((bs, H, d)).astype(np.float32)
+    u = _direction(q, w).astype(np.float32)
+    K = np.repeat(base[None], len(t), axis=0) + (t.astype(np.float32)[:, None, None, None]
+                                                 * u[None, None])
+    K = K.reshape(len(t) * bs, H, d).astype(np.float32)
+    V = rng.standard_normal(K.shape).astype(np.float32)
+    return K, V
+
+
+def _run(w, K, V, q, groups):
+    cfg = feed_gpu.config_of(w)
+    table = torch.from_numpy(gen.block_table(w))
+    cache = SplaDecodeCache(cfg, 1, table, w.num_phys_blocks, device="cuda")
+    for s in range(0, K.shape[0], CHUNK):
+        k = torch.from_numpy(np.ascontiguousarray(K[None, s:s + CHUNK])).cuda()
+        v = torch.from_numpy(np.ascontiguousarray(V[None, s:s + CHUNK])).cuda()
+        cache.append(k, v)
+    gamma = gen.gamma(w)
+    qt = torch.from_numpy(q).cuda()
+    out, sel, osp, orl = cache.new_outputs(debug=True)
+    cache.decode(qt, torch.from_numpy(gamma).cuda(), out, sel, osp, orl)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    res = dict(out=out.cpu().numpy(), sel=sel.cpu().numpy(), o_sparse=osp.cpu().numpy(),
+               o_rla=orl.cpu().numpy())
+    oc = so.OracleCache(ofeed.params_of(w), 1, groups)
+    for (b, h) in groups:
+        oc.append_group(b, h, K[:, h].astype(np.float64), V[:, h].astype(np.float64))
+    return res, oc, gamma
+
+
+@pytest.mark.parametrize("n_blocks", [150, 1200])
+def test_exact_ties_taken_in_block_order(n_blocks):
+    """Two score classes: every block of the higher one, then the lowest-indexed of the
+    lower one. 150 blocks keep the tied class under the candidate cap; 1200 push it
+    past it, through the key-space refinement down to a single repeated key."""
+    w = _workload(n_blocks)
+    q = gen.query(w, 0)
+    rng = np.random.default_rng(5)
+    hi = rng.choice(np.arange(1, n_blocks - 1), size=10, replace=False)
+    t = np.zeros(n_blocks)
+    t[hi] = 1.0
+    K, V = _keys(w, t, q, seed=11)
+    groups = [(0, 0), (0, 5)]
+    res, oc, gamma = _run(w, K, V, q, groups)
+    for (b, h) in groups:
+        for hq in range(h * w.group, (h + 1) * w.group):
+            # the class offset raises this head's estimate only if q_hq points along u
+            lift = float(q[0, hq] @ _direction(q, w)[h])
+            top = set(hi.tolist()) if lift > 0 else None
+            sel = set(int(x) for x in res["sel"][0, hq] if x >= 0)
+            forced = {0, n_blocks - 1}
+            assert forced <= sel
+            pool = sorted(set(range(1, n_blocks - 1)) - (top or set()))
+            if top is not None:
+                want = forced | top | set(pool[:w.top_k - len(top)])
+            else:
+                lows = set(range(1, n_blocks - 1)) - set(hi.tolist())
+                want = forced | set(sorted(lows)[:w.top_k])
+            assert sel == want, (hq, sorted(sel ^ want)[:8])
+            parity.compare_head({k: v[0, hq] for k, v in res.items()}, oc, q, gamma, 0, hq, "f32")
+
+
+def test_crowded_bucket_distinct_scores():
+    """Distinct scores 1e-3 apart packed into two of the 2048 value buckets by far
+    outliers on both sides: the selection must still be the exact top-k."""
+    n_blocks = 1200
+    w = _workload(n_blocks)
+    q = gen.query(w, 0)
+    rng = np.random.default_rng(7)
+    t = 1e-3 * rng.permutation(n_blocks).astype(np.float64)
+    t[rng.choice(np.arange(1, n_blocks - 1), size=5, replace=False)] = 1000.0
+    t[rng.choice(np.arange(1, n_blocks - 1), size=1)] = -1000.0
+    K, V = _keys(w, t, q, seed=3)
+    groups = [(0, 1), (0, 6)]
+    res, oc, gamma = _run(w, K, V, q, groups)
+    for (b, h) in groups:
+        for hq in range(h * w.group, (h + 1) * w.group):
+            st = parity.compare_head({k: v[0, hq] for k, v in res.items()}, oc, q, gamma, 0, hq,
+                                     "f32")
+            assert st["ties"] == 0
