@@ -450,6 +450,7 @@ constexpr int kCandCap = 256;
 constexpr uint32_t kMark = 0xffffffffu;     // a selected key (only a NaN score maps here)
 constexpr int kWordsPerThread = SPLA_MAX_BLOCKS_PER_SEQ / 32 / kSelThreads;
 static_assert(kWordsPerThread * 32 * kSelThreads == SPLA_MAX_BLOCKS_PER_SEQ, "bitset words per thread");
+static_assert(SPLA_MAX_BLOCKS_PER_SEQ / kSelThreads <= 64, "candidate rounds fit a 64-bit mask");
 
 // The float a key was made from (the inverse of ordered_key).
 __device__ __forceinline__ float key_value(uint32_t k) {
@@ -534,6 +535,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem_sel);        // [mbp padded]
     __shared__ int hist[kBins];
     __shared__ int wpre[SPLA_MAX_BLOCKS_PER_SEQ / 32];             // per-word counts, then prefixes
+    __shared__ uint32_t wword[SPLA_MAX_BLOCKS_PER_SEQ / 32];       // the bitset words
     __shared__ uint32_t cand_key[kCandCap];
     __shared__ int cand_idx[kCandCap];
     __shared__ __align__(16) unsigned long long cand_c[kCandCap];   // key << 32 | ~index
@@ -548,10 +550,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
     // the decode kernels launch only now: before their own wait they may read what
     // the scoring kernel wrote (it has completed)
     pdl_trigger();
+    const float* sc = scores + ((int64_t)b * c.hq + hq) * c.mbp;
+    // the first batch of score loads goes out with the length load, bounded by the
+    // capacity (entries past the sequence's blocks are loaded and ignored)
+    constexpr int kKeyBatch = 8;
+    float x0[kKeyBatch];
+#pragma unroll
+    for (int u = 0; u < kKeyBatch; ++u) {
+        const int j = tid + u * kSelThreads;
+        x0[u] = (j < c.mbp) ? __ldcg(sc + j) : 0.f;
+    }
     int32_t L = c.lens[b];
     L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + c.bs - 1) / c.bs;
-    const float* sc = scores + ((int64_t)b * c.hq + hq) * c.mbp;
     // block j belongs to thread j % kSelThreads; rounds of kSelThreads consecutive blocks
     const int rounds = (nb + kSelThreads - 1) / kSelThreads;
 
@@ -564,13 +575,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
 
     // ---- keys, their range, and cleared bucket counters
     uint32_t lmin = 0xffffffffu, lmax = 0u;
-    constexpr int kKeyBatch = 8;                    // score loads in flight before any key is formed
+    // kKeyBatch score loads in flight before any key is formed
     for (int j0 = tid; j0 < nb; j0 += kKeyBatch * kSelThreads) {
         float x[kKeyBatch];
 #pragma unroll
         for (int u = 0; u < kKeyBatch; ++u) {
             const int j = j0 + u * kSelThreads;
-            x[u] = (j < nb) ? __ldcg(sc + j) : 0.f;
+            x[u] = (j0 == tid) ? x0[u] : ((j < nb) ? __ldcg(sc + j) : 0.f);
         }
 #pragma unroll
         for (int u = 0; u < kKeyBatch; ++u) {
@@ -608,9 +619,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
             auto fbin = [&](uint32_t k) {
                 return min(kBins - 1, max(0, (int)((key_value(k) - fmin) * scl)));
             };
-            for (int j = tid; j < nb; j += kSelThreads) {
-                const uint32_t k = keys[j];
-                if (k) atomicAdd(&hist[fbin(k)], 1);
+            // four keys per step, their loads and bucket arithmetic independent
+            for (int j0 = tid; j0 < nb; j0 += 4 * kSelThreads) {
+                uint32_t kk[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = j0 + u * kSelThreads;
+                    kk[u] = j < nb ? keys[j] : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (kk[u]) atomicAdd(&hist[fbin(kk[u])], 1);
             }
             __syncthreads();
             // suffix scan from the top bucket; thread t covers reversed buckets [4t, 4t+4)
@@ -636,29 +655,34 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
             __syncthreads();
             const int bstar = s_bstar, krem = s_krem;
             if (s_cnt <= kCandCap) {
-                // everything above the bucket is selected; the bucket's keys are candidates
-                for (int r = 0; r < rounds; ++r) {
-                    const int j = r * kSelThreads + tid;
-                    bool in = false;
-                    if (j < nb) {
-                        const uint32_t k = keys[j];
-                        if (k) {
-                            const int bb = fbin(k);
-                            if (bb > bstar) keys[j] = kMark;
-                            in = bb == bstar;
+                // everything above the bucket is selected; the bucket's keys are
+                // candidates, recorded per thread (bit r: round r) and placed by a scan
+                unsigned long long cmask = 0ull;
+                for (int r0 = 0; r0 < rounds; r0 += 4) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int r = r0 + u, j = r * kSelThreads + tid;
+                        if (r < rounds && j < nb) {
+                            const uint32_t k = keys[j];
+                            if (k) {
+                                const int bb = fbin(k);
+                                if (bb > bstar) keys[j] = kMark;
+                                else if (bb == bstar) cmask |= 1ull << r;
+                            }
                         }
                     }
-                    const uint32_t m = __ballot_sync(0xffffffffu, in);
-                    int base = 0;
-                    if (lane == 0 && m) base = atomicAdd(&s_ncand, __popc(m));
-                    base = __shfl_sync(0xffffffffu, base, 0);
-                    if (in) {
-                        const int p = base + __popc(m & ((1u << lane) - 1u));
-                        if (p < kCandCap) { cand_key[p] = keys[j]; cand_idx[p] = j; }
-                    }
+                }
+                int ncnd;
+                int p = block_excl_scan(__popcll(cmask), tmp, &ncnd);
+                while (cmask) {
+                    const int r = __ffsll((long long)cmask) - 1;
+                    cmask &= cmask - 1ull;
+                    const int j = r * kSelThreads + tid;
+                    if (p < kCandCap) { cand_key[p] = keys[j]; cand_idx[p] = j; }
+                    ++p;
                 }
                 __syncthreads();
-                rank_candidates(keys, cand_key, cand_idx, cand_c, min(s_ncand, kCandCap), krem);
+                rank_candidates(keys, cand_key, cand_idx, cand_c, min(ncnd, kCandCap), krem);
                 thr = kMark;
             } else {
                 // key range of the crowded bucket, then key-space refinement inside it
@@ -779,14 +803,24 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
     // ---- flags -> bitset words (one ballot per 32 consecutive blocks), then list positions
     uint32_t* hb = bits + ((int64_t)b * c.hq + hq) * nw;
     const int nwu = (nb + 31) >> 5;
-    for (int r = 0; r < rounds; ++r) {
-        const int j = r * kSelThreads + tid;
-        const bool sel = j < nb && (take_all || forced(j) || (unsigned long long)keys[j] >= thr);
-        const uint32_t word = __ballot_sync(0xffffffffu, sel);
-        const int wi = r * kSelWarps + warp;
-        if (lane == 0 && wi < nwu) {
-            hb[wi] = word;
-            wpre[wi] = __popc(word);
+    for (int r0 = 0; r0 < rounds; r0 += 4) {
+        bool sel[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = r0 + u, j = r * kSelThreads + tid;
+            sel[u] = r < rounds && j < nb &&
+                     (take_all || forced(j) || (unsigned long long)keys[j] >= thr);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = r0 + u;
+            const uint32_t word = __ballot_sync(0xffffffffu, sel[u]);
+            const int wi = r * kSelWarps + warp;
+            if (lane == 0 && r < rounds && wi < nwu) {
+                hb[wi] = word;
+                wword[wi] = word;
+                wpre[wi] = __popc(word);
+            }
         }
     }
     __syncthreads();
@@ -815,7 +849,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
             const int j = r * kSelThreads + tid;
             const int wi = r * kSelWarps + warp;
             if (wi < nwu) {
-                const uint32_t word = hb[wi];
+                const uint32_t word = wword[wi];
                 if ((word >> lane) & 1u) {
                     const int pos = wpre[wi] + __popc(word & ((1u << lane) - 1u));
                     if (pos < kcap) out[pos] = j;
