@@ -296,50 +296,72 @@ __device__ __forceinline__ int union_share_warp(const int32_t* trow, int num_phy
 }
 
 // ------------------------------------------------------------------ combine
-// One CTA per (sequence, query head), thread j owns output column j. Every
-// thread issues its loads (the splits' acc[j] and N~[j], up to 32 splits at a
-// time, the readout N[j]) before any of them is needed; the record headers go
-// through shared memory. Launched right behind the decode kernel
-// (programmatic dependent launch), it waits for it.
-constexpr int kCombChunk = 32;
+// One CTA of 16 warps per (sequence, query head). Warp w takes the splits
+// w, w + 16, ...: lane l holds columns [l d/32, (l+1) d/32) of their acc and N~
+// (vector loads), so up to 64 splits' records are in flight in one round trip
+// together with the headers and the readout N, D; the warps' partial sums meet
+// in shared memory. Launched right behind the decode kernel (programmatic
+// dependent launch), it waits for it.
+constexpr int kCombThreads = 512;
+constexpr int kCombWarps = kCombThreads / 32;
+constexpr int kCombPerWarp = 4;                 // splits per warp per round trip
 
-template <typename T>
-__global__ void __launch_bounds__(128) combine_kernel(CacheView c, const DecodeArgs a) {
+template <int D> struct CombVec;
+template <> struct CombVec<128> {
+    static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(p));
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    }
+};
+template <> struct CombVec<64> {
+    static __device__ __forceinline__ void load(const float* p, float (&v)[2]) {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(p));
+        v[0] = x.x; v[1] = x.y;
+    }
+};
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(CacheView c, const DecodeArgs a) {
+    constexpr int CPL = D / 32;                 // columns per lane
     extern __shared__ __align__(16) float smem_comb[];
-    const int d = c.d, G = c.group, REC = rec_floats(d), ns = a.nsplit;
+    const int G = c.group, ns = a.nsplit;
+    constexpr int REC = 2 * D + 4;
     const int b = blockIdx.x / c.hq, hq = blockIdx.x % c.hq;
     const int h = hq / G, g = hq % G;
-    const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
-    float* hdr = smem_comb;                 // [ns][4]: m, l, D~
-    float* fac = hdr + 4 * ns;              // [ns]
-    __shared__ float s_M, s_l, s_dt, s_D, s_red[4];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float* hdr = smem_comb;                     // [ns][4]: m, l, D~
+    float* fac = hdr + 4 * ns;                  // [ns]
+    __shared__ __align__(16) float s_po[kCombWarps][D], s_pn[kCombWarps][D];
+    __shared__ float s_M, s_l, s_dt, s_D, s_red[D / 32];
     pdl_wait();
+    const float* recs = a.part + (((int64_t)b * c.hkv + h) * ns * G + g) * REC;   // split s at s*G*REC
+    const float* gr = a.gread + (((int64_t)b * c.hkv + h) * a.nrd * G + g) * (D + 4);
+    for (int s = tid; s < ns; s += kCombThreads)
+        reinterpret_cast<float4*>(hdr)[s] = __ldcg(reinterpret_cast<const float4*>(recs + (int64_t)s * G * REC));
+    // this warp's first splits, in flight with the headers
+    float acc[kCombPerWarp][CPL], ntl[kCombPerWarp][CPL];
+#pragma unroll
+    for (int u = 0; u < kCombPerWarp; ++u) {
+        const int s = warp + u * kCombWarps;
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) acc[u][e] = ntl[u][e] = 0.f;
+        if (s < ns) {
+            const float* r = recs + (int64_t)s * G * REC + 4 + lane * CPL;
+            CombVec<D>::load(r, acc[u]);
+            CombVec<D>::load(r + D, ntl[u]);
+        }
+    }
+    float Nj = 0.f, Dg = 0.f;
+    if (tid < D)
+        for (int p = 0; p < a.nrd; ++p) {          // the readout's row-range parts add
+            Nj += __ldcg(gr + (int64_t)p * G * (D + 4) + tid);
+            if (tid == 0) Dg += __ldcg(gr + (int64_t)p * G * (D + 4) + D);
+        }
+    if (tid == 0) s_D = Dg;
+    const int nsel = a.nsel[(int64_t)b * c.hq + hq];
     int32_t L = c.lens[b];
     L = max(0, min(L, c.mbp * c.bs));
     const int nb = (L + c.bs - 1) / c.bs;
-    const float* recs = a.part + (((int64_t)b * c.hkv + h) * ns * G + g) * REC;   // split s at s*G*REC
-    const float* gr = a.gread + (((int64_t)b * c.hkv + h) * a.nrd * G + g) * (d + 4);
-    for (int s = j; s < ns; s += blockDim.x)
-        reinterpret_cast<float4*>(hdr)[s] = __ldcg(reinterpret_cast<const float4*>(recs + (int64_t)s * G * REC));
-    float Nj = 0.f, Dg = 0.f;
-    for (int p = 0; p < a.nrd; ++p) {              // the readout's row-range parts add
-        Nj += __ldcg(gr + (int64_t)p * G * (d + 4) + j);
-        if (j == 0) Dg += __ldcg(gr + (int64_t)p * G * (d + 4) + d);
-    }
-    if (j == 0) s_D = Dg;
-    const int nsel = a.nsel[(int64_t)b * c.hq + hq];
-    // first chunk of columns in flight while the headers are reduced
-    float acc_v[kCombChunk], ntl_v[kCombChunk];
-#pragma unroll
-    for (int s = 0; s < kCombChunk; ++s) {
-        acc_v[s] = 0.f;
-        ntl_v[s] = 0.f;
-        if (s < ns) {
-            const float* r = recs + (int64_t)s * G * REC;
-            acc_v[s] = __ldcg(r + 4 + j);
-            ntl_v[s] = __ldcg(r + 4 + d + j);
-        }
-    }
     __syncthreads();
     if (warp == 0) {
         float M = -SPLA_INF;
@@ -357,47 +379,82 @@ __global__ void __launch_bounds__(128) combine_kernel(CacheView c, const DecodeA
         if (lane == 0) { s_M = M; s_l = l; s_dt = dt; }
     }
     __syncthreads();
-    float o = 0.f, nt = 0.f;
+    float o[CPL], nt[CPL];
 #pragma unroll
-    for (int s = 0; s < kCombChunk; ++s)
+    for (int e = 0; e < CPL; ++e) o[e] = nt[e] = 0.f;
+#pragma unroll
+    for (int u = 0; u < kCombPerWarp; ++u) {
+        const int s = warp + u * kCombWarps;
         if (s < ns) {
-            o = fmaf(acc_v[s], fac[s], o);
-            nt += ntl_v[s];
-        }
-    for (int s0 = kCombChunk; s0 < ns; s0 += kCombChunk) {
+            const float f = fac[s];
 #pragma unroll
-        for (int u = 0; u < kCombChunk; ++u) {
-            acc_v[u] = 0.f;
-            ntl_v[u] = 0.f;
-            if (s0 + u < ns) {
-                const float* r = recs + (int64_t)(s0 + u) * G * REC;
-                acc_v[u] = __ldcg(r + 4 + j);
-                ntl_v[u] = __ldcg(r + 4 + d + j);
+            for (int e = 0; e < CPL; ++e) {
+                o[e] = fmaf(acc[u][e], f, o[e]);
+                nt[e] += ntl[u][e];
             }
         }
-#pragma unroll
-        for (int u = 0; u < kCombChunk; ++u)
-            if (s0 + u < ns) {
-                o = fmaf(acc_v[u], fac[s0 + u], o);
-                nt += ntl_v[u];
-            }
     }
-    const float lsum = s_l, Dr = s_D - s_dt;
-    const bool off = a.no_rla || nsel >= nb || !(Dr > 0.f) || L == 0;
-    const float osp = (lsum > 0.f) ? o / lsum : 0.f;
-    const float orl = off ? 0.f : (Nj - nt) / Dr;
-    // RMS of o_rla over the head dimension
-    float sq = warp_sum(orl * orl);
-    if (lane == 0) s_red[warp] = sq;
+    // more than kCombWarps * kCombPerWarp splits: further round trips
+    for (int s0 = kCombWarps * kCombPerWarp; s0 < ns; s0 += kCombWarps * kCombPerWarp) {
+#pragma unroll
+        for (int u = 0; u < kCombPerWarp; ++u) {
+            const int s = s0 + warp + u * kCombWarps;
+#pragma unroll
+            for (int e = 0; e < CPL; ++e) acc[u][e] = ntl[u][e] = 0.f;
+            if (s < ns) {
+                const float* r = recs + (int64_t)s * G * REC + 4 + lane * CPL;
+                CombVec<D>::load(r, acc[u]);
+                CombVec<D>::load(r + D, ntl[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kCombPerWarp; ++u) {
+            const int s = s0 + warp + u * kCombWarps;
+            if (s < ns) {
+                const float f = fac[s];
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    o[e] = fmaf(acc[u][e], f, o[e]);
+                    nt[e] += ntl[u][e];
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) {
+        s_po[warp][lane * CPL + e] = o[e];
+        s_pn[warp][lane * CPL + e] = nt[e];
+    }
     __syncthreads();
-    sq = 0.f;
-    for (int w = 0; w < (d + 31) / 32; ++w) sq += s_red[w];
-    const float inv = rsqrtf(sq / d + a.eps);
-    const int64_t oi = ((int64_t)b * c.hq + hq) * d + j;
-    const float gm = a.gamma ? a.gamma[(int64_t)hq * d + j] : 1.f;
-    static_cast<T*>(a.out)[oi] = from_f<T>(osp + gm * orl * inv);
-    if (a.o_sp) a.o_sp[oi] = osp;
-    if (a.o_rl) a.o_rl[oi] = orl;
+    // thread j < D finishes column j
+    float osp = 0.f, orl = 0.f;
+    if (tid < D) {
+        float ot = 0.f, ntt = 0.f;
+#pragma unroll
+        for (int w = 0; w < kCombWarps; ++w) {
+            ot += s_po[w][tid];
+            ntt += s_pn[w][tid];
+        }
+        const float lsum = s_l, Dr = s_D - s_dt;
+        const bool off = a.no_rla || nsel >= nb || !(Dr > 0.f) || L == 0;
+        osp = (lsum > 0.f) ? ot / lsum : 0.f;
+        orl = off ? 0.f : (Nj - ntt) / Dr;
+        // RMS of o_rla over the head dimension
+        const float sq = warp_sum(orl * orl);
+        if (lane == 0) s_red[warp] = sq;
+    }
+    __syncthreads();
+    if (tid < D) {
+        float sq = 0.f;
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) sq += s_red[w];
+        const float inv = rsqrtf(sq / D + a.eps);
+        const int64_t oi = ((int64_t)b * c.hq + hq) * D + tid;
+        const float gm = a.gamma ? a.gamma[(int64_t)hq * D + tid] : 1.f;
+        static_cast<T*>(a.out)[oi] = from_f<T>(osp + gm * orl * inv);
+        if (a.o_sp) a.o_sp[oi] = osp;
+        if (a.o_rl) a.o_rl[oi] = orl;
+    }
 }
 
 // ------------------------------------------------------------------ bf16 tensor-core kernel
@@ -974,10 +1031,14 @@ cudaError_t launch_decode_simt(const CacheView& c, int dtype, const DecodeArgs& 
 
 cudaError_t launch_combine(const CacheView& c, int dtype, const DecodeArgs& a, cudaStream_t s) {
     const size_t smem = (size_t)5 * a.nsplit * sizeof(float);
-    const dim3 grid(c.batch * c.hq), block(c.d);
-    if (dtype == SPLA_BF16)
-        return launch_pdl(combine_kernel<__nv_bfloat16>, grid, block, smem, s, c, a);
-    return launch_pdl(combine_kernel<float>, grid, block, smem, s, c, a);
+    const dim3 grid(c.batch * c.hq), block(kCombThreads);
+    if (c.d == 128)
+        return dtype == SPLA_BF16
+            ? launch_pdl(combine_kernel<128, __nv_bfloat16>, grid, block, smem, s, c, a)
+            : launch_pdl(combine_kernel<128, float>, grid, block, smem, s, c, a);
+    return dtype == SPLA_BF16
+        ? launch_pdl(combine_kernel<64, __nv_bfloat16>, grid, block, smem, s, c, a)
+        : launch_pdl(combine_kernel<64, float>, grid, block, smem, s, c, a);
 }
 
 }  // namespace spla

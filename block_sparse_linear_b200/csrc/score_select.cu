@@ -443,14 +443,12 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
 }
 
 // ------------------------------------------------------------------ selection
-constexpr int kSelThreads = 512;
-constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kCandCap = 256;
 constexpr uint32_t kMark = 0xffffffffu;     // a selected key (only a NaN score maps here)
-constexpr int kWordsPerThread = SPLA_MAX_BLOCKS_PER_SEQ / 32 / kSelThreads;
-static_assert(kWordsPerThread * 32 * kSelThreads == SPLA_MAX_BLOCKS_PER_SEQ, "bitset words per thread");
-static_assert(SPLA_MAX_BLOCKS_PER_SEQ / kSelThreads <= 64, "candidate rounds fit a 64-bit mask");
+// threads per head: 512, or 1024 once a sequence can hold more than 4096 blocks
+constexpr int kSelThreadsLong = 1024;
+constexpr int kSelLongBlocks = 4096;
 
 // The float a key was made from (the inverse of ordered_key).
 __device__ __forceinline__ float key_value(uint32_t k) {
@@ -491,14 +489,14 @@ __device__ int block_excl_scan(int v, int* tmp, int* total) {
 __device__ __forceinline__ void rank_candidates(uint32_t* keys, const uint32_t* cand_key,
                                                 const int* cand_idx, unsigned long long* cand_c,
                                                 int nc, int krem) {
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, nt = blockDim.x;
     const int ncp = (nc + 7) & ~7;
-    for (int i = tid; i < ncp; i += kSelThreads)
+    for (int i = tid; i < ncp; i += nt)
         cand_c[i] = (i < nc) ? (((unsigned long long)cand_key[i] << 32) |
                                 (uint32_t)~(uint32_t)cand_idx[i])
                              : 0ull;
     __syncthreads();
-    for (int i = tid; i < nc; i += kSelThreads) {
+    for (int i = tid; i < nc; i += nt) {
         const unsigned long long mine = cand_c[i];
         int rank = 0;
         // eight candidates per step, their loads in flight together
@@ -526,11 +524,18 @@ __device__ __forceinline__ void rank_candidates(uint32_t* keys, const uint32_t* 
 //              bucket) buckets linear in key space, narrowed pass by pass.
 // Every step that reads what another warp wrote is one barrier apart; no loop
 // carries a dependency through shared memory.
-__global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int top_k, int n_sink,
-                                                             int n_local, const float* scores,
-                                                             uint32_t* bits, int nw,
-                                                             int32_t* nsel, int32_t* sel_idx,
-                                                             int kcap) {
+template <int NT>
+__global__ void __launch_bounds__(NT) select_kernel(CacheView c, int top_k, int n_sink,
+                                                    int n_local, const float* scores,
+                                                    uint32_t* bits, int nw, int32_t* nsel,
+                                                    int32_t* sel_idx, int kcap) {
+    constexpr int kSelThreads = NT;
+    constexpr int kSelWarps = NT / 32;
+    constexpr int kWordsPerThread = SPLA_MAX_BLOCKS_PER_SEQ / 32 / NT;
+    constexpr int BPT = kBins / NT;             // histogram buckets per thread in the scans
+    static_assert(kWordsPerThread * 32 * NT == SPLA_MAX_BLOCKS_PER_SEQ, "bitset words per thread");
+    static_assert(SPLA_MAX_BLOCKS_PER_SEQ / NT <= 64, "candidate rounds fit a 64-bit mask");
+    static_assert(BPT * NT == kBins, "buckets per thread");
     extern __shared__ __align__(16) unsigned char smem_sel[];
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem_sel);        // [mbp padded]
     __shared__ int hist[kBins];
@@ -632,20 +637,20 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
                     if (kk[u]) atomicAdd(&hist[fbin(kk[u])], 1);
             }
             __syncthreads();
-            // suffix scan from the top bucket; thread t covers reversed buckets [4t, 4t+4)
-            int local[4], lsum = 0;
+            // suffix scan from the top bucket; thread t covers reversed buckets [BPT t, BPT t + BPT)
+            int local[BPT], lsum = 0;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                local[u] = hist[kBins - 1 - (4 * tid + u)];
+            for (int u = 0; u < BPT; ++u) {
+                local[u] = hist[kBins - 1 - (BPT * tid + u)];
                 lsum += local[u];
             }
             const int before = block_excl_scan(lsum, tmp, nullptr);
             if (before < top_k && before + lsum >= top_k) {
                 int acc = before;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < BPT; ++u) {
                     if (acc < top_k && acc + local[u] >= top_k) {
-                        s_bstar = kBins - 1 - (4 * tid + u);
+                        s_bstar = kBins - 1 - (BPT * tid + u);
                         s_krem = top_k - acc;        // still to take from the bucket
                         s_cnt = local[u];
                     }
@@ -726,10 +731,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
                     if (k >= lo && k < hi) atomicAdd(&hist[(int)((k - lo) >> shift)], 1);
                 }
                 __syncthreads();
-                int local[4], lsum = 0;
+                int local[BPT], lsum = 0;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int r = 4 * tid + u;
+                for (int u = 0; u < BPT; ++u) {
+                    const int r = BPT * tid + u;
                     local[u] = (r < nbins) ? hist[nbins - 1 - r] : 0;
                     lsum += local[u];
                 }
@@ -738,9 +743,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(CacheView c, int to
                 if (before < krem && before + lsum >= krem) {
                     int acc = before;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < BPT; ++u) {
                         if (acc < krem && acc + local[u] >= krem) {
-                            const int bst = nbins - 1 - (4 * tid + u);
+                            const int bst = nbins - 1 - (BPT * tid + u);
                             const unsigned long long nlo = lo + ((unsigned long long)bst << shift);
                             unsigned long long nhi = lo + ((unsigned long long)(bst + 1) << shift);
                             if (nhi > hi) nhi = hi;
@@ -899,12 +904,13 @@ cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local
                           const float* scores, uint32_t* bits, int nw, int32_t* nsel,
                           int32_t* sel_idx, int kcap, cudaStream_t s) {
     const size_t smem = (size_t)((c.mbp + 31) / 32) * 32 * sizeof(uint32_t);
+    const bool lng = c.mbp > kSelLongBlocks;
+    auto kern = lng ? select_kernel<kSelThreadsLong> : select_kernel<512>;
     // static plus dynamic shared memory may pass the 48 KiB default
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(select_kernel, dim3(c.batch * c.hq), dim3(kSelThreads), smem, s, c, top_k,
-                      n_sink, n_local, scores, bits, nw, nsel, sel_idx, kcap);
+    return launch_pdl(kern, dim3(c.batch * c.hq), dim3(lng ? kSelThreadsLong : 512), smem, s, c,
+                      top_k, n_sink, n_local, scores, bits, nw, nsel, sel_idx, kcap);
 }
 
 }  // namespace spla
