@@ -229,69 +229,72 @@ __device__ __noinline__ int union_share(const int32_t* trow, int num_phys, int G
     return n;
 }
 
-// The same share built by one warp, 32 words at a time (lane l takes word
-// w0 + l): a first sweep counts the union, a second places every word by a
-// shuffle scan and each lane extracts its own word's blocks, head masks and
-// physical blocks. No CTA barrier inside, and no lane walks more than one word
-// per sweep step.
-__device__ __forceinline__ int union_share_warp(const int32_t* trow, int num_phys, int G,
-                                                const uint32_t* wbits, int ws, int nwu, int nb,
-                                                int split, int nsplit, int max_per, int32_t* blk,
-                                                int32_t* phys, uint32_t* hm, int32_t* status,
-                                                int lane) {
-    // wbits: [G][ws] words, the first nwu of each row in use
+// This CTA's share of the union of the group's G selections, built by all NT
+// threads: thread t takes consecutive words [t W, t W + W) so that union ranks run
+// in word order; one block scan of the per-thread counts gives every thread its
+// first rank, and the ranks in [u0, u1) = [split tot / nsplit, (split+1) tot / nsplit)
+// are written out in rank order (block index, head mask, physical block).
+// wbits: [G][ws] words in shared memory, the first nwu of each row in use.
+template <int NT>
+__device__ int union_share_cta(const int32_t* trow, int num_phys, int G, const uint32_t* wbits,
+                               int ws, int nwu, int nb, int split, int nsplit, int max_per,
+                               int32_t* blk, int32_t* phys, uint32_t* hm, int32_t* status,
+                               int* s_wsum) {
+    constexpr int NWARP = NT / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     auto word = [&](int w) -> uint32_t {
         uint32_t u = 0u;
         for (int g = 0; g < G; ++g) u |= wbits[g * ws + w];
         if (w == nwu - 1 && (nb & 31)) u &= (1u << (nb & 31)) - 1u;
         return u;
     };
-    int tot = 0;
-    for (int w0 = 0; w0 < nwu; w0 += 32) {
-        const int w = w0 + lane;
-        if (w < nwu) tot += __popc(word(w));
-    }
+    const int wpt = (nwu + NT - 1) / NT;
+    const int w0 = min(nwu, tid * wpt), w1 = min(nwu, w0 + wpt);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(word(w));
+    int x = cnt;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_wsum[warp] = x;
+    __syncthreads();
+    int before = x - cnt, tot = 0;
+#pragma unroll
+    for (int v = 0; v < NWARP; ++v) {
+        const int t = s_wsum[v];
+        if (v < warp) before += t;
+        tot += t;
+    }
     // the union holds at most 32768 blocks and nsplit is at most 512: 32-bit products
     const int u0 = split * tot / nsplit, u1 = (split + 1) * tot / nsplit;
-    int base = 0;
-    for (int w0 = 0; w0 < nwu && base < u1; w0 += 32) {
-        const int w = w0 + lane;
-        uint32_t u = (w < nwu) ? word(w) : 0u;
-        const int cnt = __popc(u);
-        int x = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        int r = base + x - cnt;
-        base += __shfl_sync(0xffffffffu, x, 31);
-        if (r < u1 && r + cnt > u0) {
-            while (u) {
-                const int bit = __ffs(u) - 1;
-                u &= u - 1u;
-                if (r >= u0 && r < u1 && r - u0 < max_per) {
-                    const int e = r - u0, j = (w << 5) + bit;
-                    uint32_t mask = 0u;
-                    for (int g = 0; g < G; ++g) mask |= ((wbits[g * ws + w] >> bit) & 1u) << g;
-                    int32_t p = trow[j];
-                    if (p < 0 || p >= num_phys) {
-                        // read nothing from it: no head attends to it
-                        set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
-                        p = 0;
-                        mask = 0u;
-                    }
-                    blk[e] = j;
-                    hm[e] = mask;
-                    phys[e] = p;
+    int r = before;
+    for (int w = w0; w < w1 && r < u1; ++w) {
+        uint32_t u = word(w);
+        const int cw = __popc(u);
+        if (r + cw <= u0) { r += cw; continue; }
+        while (u) {
+            const int bit = __ffs(u) - 1;
+            u &= u - 1u;
+            if (r >= u0 && r < u1 && r - u0 < max_per) {
+                const int e = r - u0, j = (w << 5) + bit;
+                uint32_t mask = 0u;
+                for (int g = 0; g < G; ++g) mask |= ((wbits[g * ws + w] >> bit) & 1u) << g;
+                int32_t p = trow[j];
+                if (p < 0 || p >= num_phys) {
+                    // read nothing from it: no head attends to it
+                    set_status(status, SPLA_DEV_BAD_BLOCK_TABLE);
+                    p = 0;
+                    mask = 0u;
                 }
-                ++r;
+                blk[e] = j;
+                hm[e] = mask;
+                phys[e] = p;
             }
+            ++r;
         }
     }
-    __syncwarp();
     return min(u1 - u0, max_per);
 }
 
@@ -489,7 +492,7 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         (reinterpret_cast<uintptr_t>(hm + a.max_per) + 15) & ~uintptr_t(15));   // [4][D]
     float* aw = qs + G4 * D;                                // [4][D]
     float* ml = aw + G4 * D;                                // [D]
-    __shared__ int s_n[2], s_abort;
+    __shared__ int s_n[2], s_abort, s_wsum[Cfg::THREADS / 32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.y / c.hkv, h = blockIdx.y % c.hkv, split = blockIdx.x;
@@ -555,16 +558,15 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         }
     }
     pdl_wait();
-    // the group's selections (one round of loads by every thread), then the producer
-    // warp alone builds this CTA's share of their union
+    // the group's selections (one round of loads by every thread), then every
+    // thread builds its words' part of this CTA's share of their union
     if (nb > 0) {
         stage_bits_vec(a.bits, a.nw, c.hq, G, b, h, wbits, tid, blockDim.x);
         __syncthreads();
-        if (warp == NCW) {
-            const int n = union_share_warp(trow, c.num_phys, G, wbits, a.nw, nwu, nb, split,
-                                           nsplit, a.max_per, blk, phys, hm, a.status, lane);
-            if (lane == 0) s_n[0] = n;
-        }
+        const int n = union_share_cta<Cfg::THREADS>(trow, c.num_phys, G, wbits, a.nw, nwu, nb,
+                                                    split, nsplit, a.max_per, blk, phys, hm,
+                                                    a.status, s_wsum);
+        if (tid == 0) s_n[0] = n;
     } else if (tid == 0) {
         s_n[0] = 0;
     }
