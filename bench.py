@@ -411,7 +411,9 @@ def oracle_sample(w, budget_s: float, steps: int = None):
     oc = ofeed.build(w, groups=[(0, 0)])
     gamma = gen.gamma(w)
     units, t_spent, n = 0, 0.0, 0
-    while (steps is None and t_spent < budget_s) or (steps is not None and n < steps):
+    # every step appends one token: stay inside the capacity reserved past the prefix
+    cap = w.extra_tokens
+    while n < cap and ((steps is None and t_spent < budget_s) or (steps is not None and n < steps)):
         k, v = gen.step_tokens(w, n)
         q = gen.query(w, n)
         t0 = time.perf_counter()

@@ -63,3 +63,16 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_0():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_oracle_sample_stays_inside_the_reserved_capacity():
+    """The CPU baseline appends one token per step: it stops at the workload's reserved
+    capacity however much time budget is left."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from workloads import gen
+    w = gen.scaled("cfg1", context_lens=(256,), extra_tokens=8)
+    *_, n = bench.oracle_sample(w, budget_s=60.0)
+    assert n == 8
+    *_, n = bench.oracle_sample(w, 0.0, steps=20)
+    assert n == 8
