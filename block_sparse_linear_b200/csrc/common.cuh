@@ -187,6 +187,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_
         :: "r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y) : "memory");
 }
 
+// L2 prefetch of one tile of a 2-D tensor map (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];"
+                 :: "l"(tmap), "r"(x), "r"(y) : "memory");
+}
+
 // Bring a kernel-parameter tensor map into the TMA unit's descriptor cache.
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(tmap) : "memory");

@@ -141,6 +141,20 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
 
     pdl_trigger();
     if (threadIdx.x == 0) prefetch_tmap(&tstats);
+    // Before the dependency wait, warm L2 with the first stage of this pair's first
+    // score item (its two boxes). A prefetch only: the copies that use the data go out
+    // after the wait and read L2, which holds whatever the append kernels wrote. Those
+    // first copies then hit L2 instead of queueing behind every pair's first request.
+    if (leader) {
+        for (int i = wp; i < nitems; i += NP) {
+            if (i < nread) continue;
+            const int r = i - nread, gi = r / ntile, t = r % ntile;
+            const int y = gi * mbp + t * kTile;
+            tma_prefetch_2d(&tstats, 0, y);
+            tma_prefetch_2d(&tstats, D, y);
+            break;
+        }
+    }
     if (leader) {
         for (int s = 0; s < kScoreRing; ++s) mbar_init(&bar[s], 1);
         mbar_init(&qbar[0], 1);
