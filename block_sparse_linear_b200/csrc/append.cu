@@ -119,12 +119,13 @@ __device__ void append_block(const CacheView& c, const T* k_new, const T* v_new,
 }
 
 // Rows [8*rg, +8) of S (and the same entries of z, m) of one (sequence, KV head).
-// Warp r owns row r; lane l owns columns l, l+32, ... of that row.
+// Warp r owns row r; lane l owns columns l, l+32, ... of that row. The row's state
+// (m, z, S) and the first new token's k and v do not depend on the length or the
+// count: they are loaded together with them, so a one-token append takes one round
+// trip before its arithmetic.
 template <typename T>
 __device__ void append_rows(const CacheView& c, const T* k_new, const T* v_new,
                             const int32_t* n_new, int32_t max_new, int b, int h, int rg) {
-    int32_t L0, n;
-    if (!append_ok(c, n_new, max_new, b, &L0, &n) || n == 0) return;
     const int d = c.d;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = rg * 8 + warp;
@@ -134,30 +135,42 @@ __device__ void append_rows(const CacheView& c, const T* k_new, const T* v_new,
     auto kval = [&](int t) -> float {
         return to_f(k_new[(((int64_t)b * max_new + t) * c.hkv + h) * d + row]);
     };
-    // running max of this dimension over the new tokens
-    float mx = -SPLA_INF;
-    for (int t = lane; t < n; t += 32) mx = fmaxf(mx, kval(t));
-    mx = warp_max(mx);
-    const float m_old = c.m[gidx];
-    const float m_new = fmaxf(m_old, mx);
-    const float f = (m_old == -SPLA_INF) ? 0.f : expf(m_old - m_new);
     constexpr int CPL = 4;                         // columns per lane (d <= 128)
-    float acc[CPL], tot[CPL];
+    // loads that need neither the length nor the count (max_new >= 1 here)
+    float s_old[CPL], v0[CPL];
+    const T* vr0 = v_new + (((int64_t)b * max_new) * c.hkv + h) * d;
 #pragma unroll
     for (int u = 0; u < CPL; ++u) {
         const int j = lane + 32 * u;
-        tot[u] = (j < d) ? Srow[j] * f : 0.f;
+        s_old[u] = (j < d) ? Srow[j] : 0.f;
+        v0[u] = (j < d) ? to_f(vr0[j]) : 0.f;
+    }
+    const float m_old = c.m[gidx], z_old = c.z[gidx];
+    const float k0 = kval(0);
+    int32_t L0, n;
+    if (!append_ok(c, n_new, max_new, b, &L0, &n) || n == 0) return;
+    // running max of this dimension over the new tokens
+    float mx = (lane == 0) ? k0 : -SPLA_INF;
+    for (int t = lane; t < n; t += 32)
+        if (t > 0) mx = fmaxf(mx, kval(t));
+    mx = warp_max(mx);
+    const float m_new = fmaxf(m_old, mx);
+    const float f = (m_old == -SPLA_INF) ? 0.f : expf(m_old - m_new);
+    float acc[CPL], tot[CPL];
+#pragma unroll
+    for (int u = 0; u < CPL; ++u) {
+        tot[u] = s_old[u] * f;
         acc[u] = 0.f;
     }
-    float zacc = 0.f, ztot = c.z[gidx] * f;
+    float zacc = 0.f, ztot = z_old * f;
     // new tokens, summed in chunks of 256 before joining the running total
     for (int t = 0; t < n; ++t) {
-        const float e = expf(kval(t) - m_new);
+        const float e = expf((t == 0 ? k0 : kval(t)) - m_new);
         const T* vr = v_new + (((int64_t)b * max_new + t) * c.hkv + h) * d;
 #pragma unroll
         for (int u = 0; u < CPL; ++u) {
             const int j = lane + 32 * u;
-            if (j < d) acc[u] = fmaf(e, to_f(vr[j]), acc[u]);
+            if (j < d) acc[u] = fmaf(e, t == 0 ? v0[u] : to_f(vr[j]), acc[u]);
         }
         zacc += e;
         if ((t & 255) == 255) {
