@@ -992,7 +992,6 @@ static cudaError_t launch_mma_t(const CacheView& c, const CUtensorMap& tk, const
 }
 
 // The merge area reuses the stage ring; it must fit.
-constexpr int kMaxSplit = 512;
 static_assert(2 * MmaCfg<128, 1, 2>::STAGE_BYTES >= (2 * 4 * 4 * 132 + 16 + 48) * 4, "merge area");
 static_assert(4 * MmaCfg<64, 1, 4>::STAGE_BYTES >= (2 * 4 * 4 * 68 + 16 + 48) * 4, "merge area");
 
