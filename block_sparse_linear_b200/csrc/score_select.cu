@@ -188,14 +188,26 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
 
     // ---- producer state (the leader): item, stage within it, stages issued
     int pi = next_item(wp), ps = 0, fi = 0, pk = 0;     // pk: items issued
+    // the current item's source, worked out at its first stage: the statistics row of
+    // its tile, or its part of S
+    int py = 0;
+    const float* psrc = nullptr;
     auto issue = [&]() {
         if (pi >= nitems) return;
         const int slot = fi % kScoreRing;
         unsigned char* dst = ring + slot * kScoreStage;
         if (ps == 0) {
             // the item's query rows (and m, z for a readout) on the item barrier
-            const int gi = pi < nread ? pi / RP : (pi - nread) / ntile;
-            const int b = gi / hkv, h = gi % hkv;
+            int gi;
+            if (pi < nread) {
+                gi = pi / RP;
+                psrc = c.S + (int64_t)gi * D * D + (int64_t)(pi % RP) * TS * RPS * D;
+            } else {
+                const int r = pi - nread;
+                gi = r / ntile;
+                py = gi * mbp + (r - gi * ntile) * kTile;
+            }
+            const int b = gi / hkv, h = gi - (gi / hkv) * hkv;
             const uint32_t qb = (uint32_t)(G * D * sizeof(T));
             unsigned char* ax = aux0 + (pk & 1) * S::kAuxPad;
             uint64_t* qb_bar = &qbar[pk & 1];
@@ -209,14 +221,10 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
         }
         mbar_arrive_expect_tx(&bar[slot], kScoreStage);
         if (pi < nread) {
-            const int gi = pi / RP, part = pi % RP;
-            const float* src = c.S + (int64_t)gi * D * D + ((int64_t)part * TS + ps) * RPS * D;
-            bulk_load(dst, src, kScoreStage, &bar[slot]);
+            bulk_load(dst, psrc + (int64_t)ps * RPS * D, kScoreStage, &bar[slot]);
         } else {
-            const int r = pi - nread, gi = r / ntile, t = r % ntile;
-            const int y = gi * mbp + t * kTile;
-            tma_load_2d(dst, &tstats, &bar[slot], ps * 32, y);
-            tma_load_2d(dst + kScoreStage / 2, &tstats, &bar[slot], D + ps * 32, y);
+            tma_load_2d(dst, &tstats, &bar[slot], ps * 32, py);
+            tma_load_2d(dst + kScoreStage / 2, &tstats, &bar[slot], D + ps * 32, py);
         }
         ++fi;
         if (++ps == TS) {
