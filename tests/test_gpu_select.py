@@ -69,11 +69,12 @@ def _run(w, K, V, q, groups):
     return res, oc, gamma
 
 
-@pytest.mark.parametrize("n_blocks", [150, 1200])
+@pytest.mark.parametrize("n_blocks", [150, 1200, 4200])
 def test_exact_ties_taken_in_block_order(n_blocks):
     """Two score classes: every block of the higher one, then the lowest-indexed of the
     lower one. 150 blocks keep the tied class under the candidate cap; 1200 push it
-    past it, through the key-space refinement down to a single repeated key."""
+    past it, through the key-space refinement down to a single repeated key; 4200 run
+    the same on the 1024-thread selection (more than 4096 blocks per sequence)."""
     w = _workload(n_blocks)
     q = gen.query(w, 0)
     rng = np.random.default_rng(5)
@@ -101,10 +102,11 @@ def test_exact_ties_taken_in_block_order(n_blocks):
             parity.compare_head({k: v[0, hq] for k, v in res.items()}, oc, q, gamma, 0, hq, "f32")
 
 
-def test_crowded_bucket_distinct_scores():
-    """Distinct scores 1e-3 apart packed into two of the 2048 value buckets by far
-    outliers on both sides: the selection must still be the exact top-k."""
-    n_blocks = 1200
+@pytest.mark.parametrize("n_blocks", [1200, 4200])
+def test_crowded_bucket_distinct_scores(n_blocks):
+    """Distinct scores 1e-3 apart packed into a few of the 2048 value buckets by far
+    outliers on both sides: the selection must still be the exact top-k (512 threads
+    per head at 1200 blocks, 1024 at 4200)."""
     w = _workload(n_blocks)
     q = gen.query(w, 0)
     rng = np.random.default_rng(7)
