@@ -9,16 +9,17 @@
 // Design", section 1; normalised linear attention as in its section 7.
 //
 // Grid (nsplit, batch*Hkv). Every CTA of a (sequence, KV head) group:
-//   * forms the union of the G heads' selections from their bitsets and takes
-//     an equal share of it (a union block is read once for all G heads; a head
-//     that did not select it is masked out of it);
+//   * forms the union of the G heads' selections from their bitsets (all
+//     threads, one block scan over the words) and takes an equal share of it
+//     (a union block is read once for all G heads; a head that did not select
+//     it is masked out of it);
 //   * streams its blocks' K and V tiles and accumulates, per head, the online
 //     softmax (m, l, acc = sum p v) and the kept blocks' linear-attention
 //     numerator and denominator (N~ = sum w v, D~ = sum w) with
 //     w_t = sum_i exp(q_i + m_i - c) exp(k_t,i - m_i);
 //   * writes one partial record per head: m, l, acc, N~, D~.
-// combine_kernel (one CTA per query head, launched right behind) merges the
-// head's records: log-sum-exp merge of the softmax partials,
+// combine_kernel (one CTA of 16 warps per query head, launched right behind)
+// merges the head's records: log-sum-exp merge of the softmax partials,
 // o_rla = (N - N~)/(D - D~) with the global readout N, D the scoring kernel
 // computed from S, z; RMSNorm; out = o_sparse + gamma * RMSNorm(o_rla).
 //
