@@ -154,10 +154,17 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
 
 def source_digest(fname: str) -> str:
+    """sha256/16 of a kernel source with its comments and blank lines removed: a capture
+    stays valid across comment edits, and only across those."""
     import hashlib
+    import re
     path = os.path.join(ROOT, "block_sparse_linear_b200", "csrc", fname)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(path) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def measured_traffic(workload: str, context: int, phase: str):

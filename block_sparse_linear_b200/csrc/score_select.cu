@@ -4,18 +4,20 @@
 // exp(q.kbar)(1 + 1/2 q^T diag(sigma^2) q); the blocks with the largest
 // estimates are attended exactly).
 //
-// score_kernel  persistent grid (2 CTAs of 4 warps per SM), every warp its
-//               own TMA pipeline over equal 32 KiB items: 32-block tiles of
-//               the statistics (fp64 tensor-core dot products with the means,
-//               fp32 sums of the non-negative variance terms) and row
-//               ranges of the global state S for the linear-attention readout
-//               N, D that the combine step subtracts from.
-// select_kernel grid (batch*Hq), 512 threads. Exact top-k by key-space
-//               bucketing: 2048 linear buckets over the live key range, the
-//               bucket holding the k-th key is refined until few candidates
-//               remain, which are ranked pairwise (ties -> lower block index).
-//               Writes a per-head selection bitset (warp ballots over 32
-//               consecutive blocks), the sorted block list and its length.
+// score_kernel  persistent grid (2 CTAs of 4 warp pairs per SM); every pair is
+//               its own TMA pipeline over equal 32 KiB items: 32-block tiles of
+//               the statistics (fp64 tensor-core dot products with the means and
+//               the variances) and row ranges of the global state S for the
+//               linear-attention readout N, D that the combine step subtracts
+//               from.
+// select_kernel grid (batch*Hq), 512 threads (1024 past 4096 blocks per
+//               sequence). Exact top-k: 2048 buckets linear in the score value,
+//               everything above the bucket holding the k-th key kept, that
+//               bucket's keys ranked pairwise (ties -> lower block index); a
+//               non-finite range or a crowded bucket falls back to key-space
+//               buckets refined pass by pass. Writes a per-head selection bitset
+//               (warp ballots over 32 consecutive blocks), the sorted block list
+//               and its length.
 #include "common.cuh"
 
 namespace spla {
