@@ -13,7 +13,11 @@ Acceptance, per (sequence, query head):
 o_rla and out are compared only where the RLA subtraction is well
 conditioned: kappa = max(D/(D - D~), |N|_inf/|N - N~|_inf), computed by the
 oracle in fp64, bounds how much the fp32 state's rounding is amplified. Heads
-past KAPPA_MAX are reported; o_sparse and the selection are still checked.
+past KAPPA_MAX are counted, returned with their kappa, and capped by the tests
+(ILL_CAP: none outside the 1M-token Student-t workload); o_sparse and the
+selection are still checked on them. A head whose residual denominator the GPU
+could not resolve (its o_rla set to 0 and SPLA_DEV_RLA_UNRESOLVED raised) must be
+one of them.
 """
 import numpy as np
 
@@ -22,6 +26,13 @@ from oracle import spla_oracle as so
 SEL_TIE = 1e-6
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 KAPPA_MAX = {"f32": 10.0, "bf16": 2e3}
+# Ill-conditioned heads allowed per workload (by the workload's base name). The
+# oracle's own kappa over every head (full size and test size) is at most 2 for
+# the 4K, 32K, 128K and ragged workloads; only the 1M-token workload, whose
+# heavy-tailed (Student-t) key offsets let a few blocks hold nearly all of a
+# head's linear-attention mass, has heads past KAPPA_MAX.
+ILL_CAP = {"cfg1": 0, "cfg2": 0, "cfg3": 0, "cfg4": None, "cfg5": 0}
+ILL_FRACTION_CFG4 = 0.25       # at most a quarter of the compared heads
 
 
 def bf16_ulp(x):
@@ -94,11 +105,49 @@ def compare_head(gpu: dict, oc: so.OracleCache, q, gamma, b, hq, dtype: str) -> 
     e_sp = err("o_sparse")
     assert e_sp <= tol, f"o_sparse ({b},{hq}) err {e_sp:.3g} > {tol}"
     conditioned = k <= KAPPA_MAX[dtype]
-    e_rl = e_out = None
+    # errors of every head are measured; only conditioned heads must meet the bound
+    e_rl = err("o_rla")
+    e_out = err("out")
     if conditioned:
-        e_rl = err("o_rla")
-        e_out = err("out")
         assert e_rl <= tol, f"o_rla ({b},{hq}) err {e_rl:.3g} > {tol} (kappa {k:.3g})"
         assert e_out <= tol, f"out ({b},{hq}) err {e_out:.3g} > {tol} (kappa {k:.3g})"
-    return dict(ties=ties, kappa=k, e_sparse=e_sp, e_rla=e_rl, e_out=e_out,
-                conditioned=conditioned)
+    unresolved = (not all_kept and not p.no_rla and np.all(np.asarray(gpu["o_rla"]) == 0))
+    return dict(b=b, hq=hq, ties=ties, kappa=k, e_sparse=e_sp, e_rla=e_rl, e_out=e_out,
+                conditioned=conditioned, unresolved=unresolved)
+
+
+def summary(stats) -> dict:
+    """Counts over compared heads: ill-conditioned heads with their kappa, worst errors."""
+    ill = [(s["b"], s["hq"], float(f"{s['kappa']:.3g}")) for s in stats if not s["conditioned"]]
+    cond = [s for s in stats if s["conditioned"]]
+    return dict(heads=len(stats), ties=sum(s["ties"] for s in stats), ill=len(ill),
+                ill_heads=ill,
+                max_sparse=max(s["e_sparse"] for s in stats),
+                max_rla=max((s["e_rla"] for s in cond), default=0.0),
+                max_out=max((s["e_out"] for s in cond), default=0.0),
+                unresolved=[(s["b"], s["hq"]) for s in stats if s["unresolved"]])
+
+
+def check_ill(name: str, stats, status: int, cap: int = None) -> dict:
+    """The ill-conditioned heads stay within the workload's cap (or the given one), and
+    the status word carries nothing but the unresolved-residual bit, and that only if
+    some head is ill."""
+    s = summary(stats)
+    base = name.split("-")[0]
+    if cap is None:
+        cap = ILL_CAP[base]
+        if cap is None:
+            cap = int(ILL_FRACTION_CFG4 * s["heads"])
+    assert s["ill"] <= cap, (f"{name}: {s['ill']} of {s['heads']} heads ill-conditioned "
+                             f"(cap {cap}); (b, hq, kappa): {s['ill_heads']}")
+    assert status & ~RLA_UNRESOLVED == 0, f"{name}: status {status:#x}"
+    if status & RLA_UNRESOLVED:
+        assert s["ill"] > 0, f"{name}: residual unresolved on the GPU but every head conditioned"
+    # a head the GPU left unresolved is one the oracle finds ill-conditioned
+    ill_keys = {(b, hq) for (b, hq, _) in s["ill_heads"]}
+    for bh in s["unresolved"]:
+        assert bh in ill_keys, f"{name}: head {bh} unresolved on the GPU but conditioned"
+    return s
+
+
+RLA_UNRESOLVED = 0x10

@@ -23,8 +23,8 @@ pytestmark = pytest.mark.gpu
 CHUNK = 4096          # whole blocks per append, so every block's statistics come from one call
 
 
-def _workload(n_blocks):
-    return gen.scaled("cfg3", context_lens=(64 * n_blocks,), dtype="f32", top_k=32,
+def _workload(n_blocks, dtype):
+    return gen.scaled("cfg3", context_lens=(64 * n_blocks,), dtype=dtype, top_k=32,
                       n_sink=1, n_local=1, extra_tokens=0)
 
 
@@ -44,6 +44,9 @@ def _keys(w, t, q, seed):
                                                  * u[None, None])
     K = K.reshape(len(t) * bs, H, d).astype(np.float32)
     V = rng.standard_normal(K.shape).astype(np.float32)
+    if w.dtype == "bf16":
+        # the stored values (identical offsets still give identical keys)
+        K, V = gen.round_bf16(K), gen.round_bf16(V)
     return K, V
 
 
@@ -51,31 +54,35 @@ def _run(w, K, V, q, groups):
     cfg = feed_gpu.config_of(w)
     table = torch.from_numpy(gen.block_table(w))
     cache = SplaDecodeCache(cfg, 1, table, w.num_phys_blocks, device="cuda")
+    dt = cfg.torch_dtype
     for s in range(0, K.shape[0], CHUNK):
-        k = torch.from_numpy(np.ascontiguousarray(K[None, s:s + CHUNK])).cuda()
-        v = torch.from_numpy(np.ascontiguousarray(V[None, s:s + CHUNK])).cuda()
+        k = torch.from_numpy(np.ascontiguousarray(K[None, s:s + CHUNK])).to(dt).cuda()
+        v = torch.from_numpy(np.ascontiguousarray(V[None, s:s + CHUNK])).to(dt).cuda()
         cache.append(k, v)
     gamma = gen.gamma(w)
-    qt = torch.from_numpy(q).cuda()
+    qt = torch.from_numpy(q).to(dt).cuda()
     out, sel, osp, orl = cache.new_outputs(debug=True)
     cache.decode(qt, torch.from_numpy(gamma).cuda(), out, sel, osp, orl)
     torch.cuda.synchronize()
-    assert cache.status() == 0
-    res = dict(out=out.cpu().numpy(), sel=sel.cpu().numpy(), o_sparse=osp.cpu().numpy(),
+    status = cache.status()
+    res = dict(out=out.float().cpu().numpy(), sel=sel.cpu().numpy(), o_sparse=osp.cpu().numpy(),
                o_rla=orl.cpu().numpy())
     oc = so.OracleCache(ofeed.params_of(w), 1, groups)
     for (b, h) in groups:
         oc.append_group(b, h, K[:, h].astype(np.float64), V[:, h].astype(np.float64))
-    return res, oc, gamma
+    return res, oc, gamma, status
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("n_blocks", [150, 1200, 4200])
-def test_exact_ties_taken_in_block_order(n_blocks):
+def test_exact_ties_taken_in_block_order(n_blocks, dtype):
     """Two score classes: every block of the higher one, then the lowest-indexed of the
     lower one. 150 blocks keep the tied class under the candidate cap; 1200 push it
     past it, through the key-space refinement down to a single repeated key; 4200 run
-    the same on the 1024-thread selection (more than 4096 blocks per sequence)."""
-    w = _workload(n_blocks)
+    the same with more than 4096 blocks per sequence. fp32 runs the kernel chain's
+    selection (512 or 1024 threads per head), bf16 the one-kernel path's (keys held in
+    registers by 128 threads)."""
+    w = _workload(n_blocks, dtype)
     q = gen.query(w, 0)
     rng = np.random.default_rng(5)
     hi = rng.choice(np.arange(1, n_blocks - 1), size=10, replace=False)
@@ -83,7 +90,8 @@ def test_exact_ties_taken_in_block_order(n_blocks):
     t[hi] = 1.0
     K, V = _keys(w, t, q, seed=11)
     groups = [(0, 0), (0, 5)]
-    res, oc, gamma = _run(w, K, V, q, groups)
+    res, oc, gamma, status = _run(w, K, V, q, groups)
+    stats = []
     for (b, h) in groups:
         for hq in range(h * w.group, (h + 1) * w.group):
             # the class offset raises this head's estimate only if q_hq points along u
@@ -99,25 +107,34 @@ def test_exact_ties_taken_in_block_order(n_blocks):
                 lows = set(range(1, n_blocks - 1)) - set(hi.tolist())
                 want = forced | set(sorted(lows)[:w.top_k])
             assert sel == want, (hq, sorted(sel ^ want)[:8])
-            parity.compare_head({k: v[0, hq] for k, v in res.items()}, oc, q, gamma, 0, hq, "f32")
+            stats.append(parity.compare_head({k: v[0, hq] for k, v in res.items()}, oc, q, gamma,
+                                             0, hq, dtype))
+    # selection is what this test is about: any head may be ill-conditioned, but the status
+    # may only report heads whose residual the oracle also finds below resolution
+    parity.check_ill(w.name, stats, status, cap=len(stats))
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("n_blocks", [1200, 4200])
-def test_crowded_bucket_distinct_scores(n_blocks):
-    """Distinct scores 1e-3 apart packed into a few of the 2048 value buckets by far
-    outliers on both sides: the selection must still be the exact top-k (512 threads
-    per head at 1200 blocks, 1024 at 4200)."""
-    w = _workload(n_blocks)
+def test_crowded_bucket_distinct_scores(n_blocks, dtype):
+    """Distinct scores packed into a few of the value buckets by far outliers on both
+    sides: the selection must still be the exact top-k (refinement in key space).
+    bf16 keys are spaced wider so that rounding keeps them distinct."""
+    w = _workload(n_blocks, dtype)
     q = gen.query(w, 0)
     rng = np.random.default_rng(7)
-    t = 1e-3 * rng.permutation(n_blocks).astype(np.float64)
+    t = (1e-3 if dtype == "f32" else 3e-2) * rng.permutation(n_blocks).astype(np.float64)
     t[rng.choice(np.arange(1, n_blocks - 1), size=5, replace=False)] = 1000.0
     t[rng.choice(np.arange(1, n_blocks - 1), size=1)] = -1000.0
     K, V = _keys(w, t, q, seed=3)
     groups = [(0, 1), (0, 6)]
-    res, oc, gamma = _run(w, K, V, q, groups)
+    res, oc, gamma, status = _run(w, K, V, q, groups)
+    stats = []
     for (b, h) in groups:
         for hq in range(h * w.group, (h + 1) * w.group):
             st = parity.compare_head({k: v[0, hq] for k, v in res.items()}, oc, q, gamma, 0, hq,
-                                     "f32")
-            assert st["ties"] == 0
+                                     dtype)
+            assert st["ties"] == 0 or dtype == "bf16"
+            stats.append(st)
+    # the far outliers hold nearly all linear-attention mass: heads may be ill-conditioned
+    parity.check_ill(w.name, stats, status, cap=len(stats))
