@@ -3,8 +3,9 @@
 
 One step = the whole hot path for one batch: spla_append_kv (one new token
 per sequence, updating block statistics and the linear-attention state; two
-launches) then spla_decode (four launches) (score every block -> select top-k -> exact attention over the
-kept blocks with the fused residual-linear-attention term -> combine).
+launches) then spla_decode (four launches: score every block -> select top-k ->
+exact attention over the kept blocks with the fused residual-linear-attention
+term -> combine of the splits with the residual and the RMS norm).
 
 Default workload: batch 4, 32 query / 8 KV heads, d 128, 131072-token
 contexts in 64-token blocks, top-k 32, 64 steps of append + decode (the
@@ -49,6 +50,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--also", default="cfg4",
+                    help="a second workload measured in the same run ('' for none)")
     return ap.parse_args()
 
 
@@ -214,32 +217,21 @@ def job_value(world: int, units_per_step: int, steps: int, t_ms: float) -> float
 
 
 # ----------------------------------------------------------------------------- our arm
-def run_ours(args):
+def measure(w, K, W, dev, stream, flush, rank_sync, with_e2e=True):
+    """Time K append + decode steps of workload w (after W warm-up steps): pass A gives the
+    whole-step CUDA-event time (the value); pass B zeroes the workspace's device timestamps
+    before every step and reads them after it (first CTA past its wait to last CTA exit, per
+    kernel of the decode chain), which leaves the chain's programmatic overlap untouched."""
     import torch
-    import torch.distributed as dist
 
-    from block_sparse_linear_b200 import _lib
-    from workloads import feed_gpu, gen
+    from workloads import feed_gpu
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
-    w = workload_of(args)
-    K, W = args.steps, args.warmup
     cache = feed_gpu.build_cache(w, device=dev)
-    stream = torch.cuda.current_stream(dev)
     steps = [feed_gpu.step_inputs(w, s, device=dev) for s in range(W + 2 * K)]
     gamma = torch.ones((w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
     out = torch.empty((w.batch, w.num_q_heads, w.head_dim), dtype=steps[0][2].dtype, device=dev)
     sels = torch.empty((2 * K, w.batch, w.num_q_heads, w.top_k + w.n_sink + w.n_local),
                        dtype=torch.int32, device=dev)
-    flush = L2Flush(dev)
-
     ones = torch.ones((w.batch,), dtype=torch.int32, device=dev)    # one new token per sequence
 
     def step(s, sel=None):
@@ -250,79 +242,142 @@ def run_ours(args):
     for s in range(W):
         step(s)
     torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+    rank_sync()
 
     # ---- pass A: whole-step time (the value)
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     lens0 = cache.context_lens.cpu().numpy().copy()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index or 0) as clk:
         torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
+        rank_sync()
         for i in range(K):
             flush()
             ev0[i].record(stream)
             step(W + i, sels[i])
             ev1[i].record(stream)
         torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
+        rank_sync()
     t_steps = [ev0[i].elapsed_time(ev1[i]) for i in range(K)]
-    t_total = sum(t_steps)
 
-    # ---- pass B: per-kernel events inside spla_decode (dominant-kernel roofline)
-    pe = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    for row in pe:
-        for e in row:
-            e.record(stream)                  # materialise the handles
-    torch.cuda.synchronize(dev)
+    # ---- pass B: per-kernel device timestamps of the pipelined chain
+    from block_sparse_linear_b200 import _lib
+    stamps = torch.empty((K, 4, 256, 2), dtype=torch.int64, device=dev)
+    st_view = cache.stamps()
+    _lib.spla_profile_stamps(True)
     for i in range(K):
         flush()
-        _lib.spla_profile_events([e.cuda_event for e in pe[i]])
+        st_view.zero_()
         step(W + K + i, sels[K + i])
-    _lib.spla_profile_events([])
+        stamps[i].copy_(st_view)
+    _lib.spla_profile_stamps(False)
     torch.cuda.synchronize(dev)
-    kt = np.array([[pe[i][j].elapsed_time(pe[i][j + 1]) for j in range(4)] for i in range(K)])
-    kernel_names = ["score", "select", "decode", "combine"]
+    st = stamps.cpu().numpy().view(np.uint64)
+    # per kernel: the earliest first-CTA time and the latest exit over the SM slots
+    first = (~st[:, :, :, 0].max(axis=2)).astype(np.float64)   # ns of the first CTA past its wait
+    last = st[:, :, :, 1].max(axis=2).astype(np.float64)
+    kt = (last - first) / 1e6                            # ms per kernel: score, select, decode, combine
+    chain = (last[:, 3] - first[:, 0]) / 1e6             # scoring's first CTA to the combine's last
 
-    # ---- algorithmic bytes from the selections actually made
     sel_np = sels.cpu().numpy()
-    lens_np = lens0 + 1 + np.arange(K)[:, None]          # each step appends one token first
-    by = [step_bytes(w, sel_np[i], lens_np[i]) for i in range(K)]
+    lens_a = lens0 + 1 + np.arange(K)[:, None]           # each step appends one token first
+    by_a = [step_bytes(w, sel_np[i], lens_a[i]) for i in range(K)]
     lens_b = lens0 + K + 1 + np.arange(K)[:, None]
-    byB = [step_bytes(w, sel_np[K + i], lens_b[i]) for i in range(K)]
-    status = cache.status()
+    by_b = [step_bytes(w, sel_np[K + i], lens_b[i]) for i in range(K)]
+    res = {"t_steps": t_steps, "kt": kt, "chain_ms": chain, "by_a": by_a, "by_b": by_b,
+           "status": cache.status(), "clocks": clk.summary()}
+    if with_e2e:
+        res["e2e"] = e2e_pass(w, cache, steps, W + 2 * K, K, gamma, flush, dev, stream, ones)
+    del cache
+    torch.cuda.empty_cache()
+    return res
 
-    # ---- e2e: host buffers through the same calls, copies inside the timed region
-    e2e = None
-    if not args.no_e2e:
-        e2e = e2e_pass(w, cache, steps, W + 2 * K, K, gamma, flush, dev, stream, ones)
+
+KERNEL_NAMES = ["score", "select", "decode", "combine"]
+
+
+def summarise(w, m, K, t_ms_total, hbm, peak_kind, world):
+    """Throughput and roofline figures of one measured workload."""
+    kt = m["kt"]
+    share = kt.sum(axis=0) / kt.sum()
+    dom = int(np.argmax(share))
+    dec_bytes = float(np.mean([b["kv"] for b in m["by_b"]]))
+    sco_bytes = float(np.mean([b["stats"] + b["state"] for b in m["by_b"]]))
+    dom_bytes = dec_bytes if dom == 2 else (sco_bytes if dom == 0 else 0.0)
+    dom_ms = float(np.mean(kt[:, dom]))
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    step_bytes_mean = float(np.mean([b["total"] for b in m["by_a"]]))
+    step_gbs = step_bytes_mean / (t_ms_total / K / 1e3) / 1e9
+    chain_ms = float(np.mean(m["chain_ms"]))
+    chain_gbs = float(np.mean([b["total"] for b in m["by_b"]])) / (chain_ms / 1e3) / 1e9
+    return {
+        "dom": dom, "dom_bytes": dom_bytes, "dom_ms": dom_ms, "achieved": achieved,
+        "value": job_value(world, w.batch * w.num_q_heads, K, t_ms_total),
+        "roofline": {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "achieved": round(achieved, 1),
+                     "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                     "traffic": measured_traffic(w.name, int(w.context_lens[0]), KERNEL_NAMES[dom]),
+                     "peak_kind": f"{peak_kind} hbm_gbs",
+                     "bytes_per_launch": int(dom_bytes), "ms_per_launch": round(dom_ms, 5),
+                     "timing": "device timestamps: first CTA past its dependency wait to last "
+                               "CTA exit, in the pipelined step"},
+        "step_roofline": {"bytes_per_step": int(step_bytes_mean),
+                          "kv_bytes": int(np.mean([b["kv"] for b in m["by_a"]])),
+                          "stats_bytes": int(np.mean([b["stats"] for b in m["by_a"]])),
+                          "state_bytes": int(np.mean([b["state"] for b in m["by_a"]])),
+                          "achieved_gbs": round(step_gbs, 1),
+                          "frac_of_measured_peak": round(step_gbs / hbm, 4),
+                          "frac_of_nominal_8tbs": round(step_gbs / 8000.0, 4),
+                          "decode_chain_ms": round(chain_ms, 5),
+                          "decode_chain_gbs": round(chain_gbs, 1),
+                          "decode_chain_frac_of_measured_peak": round(chain_gbs / hbm, 4)},
+        "kernels_ms": {n: round(float(np.mean(kt[:, j])), 5) for j, n in enumerate(KERNEL_NAMES)},
+        "kernel_share": {n: round(float(share[j]), 4) for j, n in enumerate(KERNEL_NAMES)},
+    }
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from workloads import gen
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def rank_sync():
+        if world > 1:
+            dist.barrier()
+
+    w = workload_of(args)
+    K, W = args.steps, args.warmup
+    stream = torch.cuda.current_stream(dev)
+    flush = L2Flush(dev)
+    m = measure(w, K, W, dev, stream, flush, rank_sync, with_e2e=not args.no_e2e)
+    t_total = sum(m["t_steps"])
+    # the other target workload (1M tokens), measured on the same box; every rank takes part
+    extra = None
+    if args.also and args.also != w.name:
+        wx = gen.get(args.also)
+        Kx = min(K, 16)
+        mx = measure(wx, Kx, W, dev, stream, flush, rank_sync, with_e2e=False)
+        extra = (wx, mx, Kx)
 
     # ---- max over ranks (the same single collective on every rank)
-    t_max, e2e_ms = max_over_ranks([t_total, e2e["ms"] if e2e is not None else 0.0], dev)
-    if e2e is not None:
-        e2e["ms"] = e2e_ms
-    units_per_step = w.batch * w.num_q_heads
-    value = job_value(world, units_per_step, K, t_max)
+    t_max, e2e_ms, tx_max = max_over_ranks(
+        [t_total, m["e2e"]["ms"] if "e2e" in m else 0.0,
+         sum(extra[1]["t_steps"]) if extra else 0.0], dev)
 
     if rank == 0:
         hbm, peak_kind = peaks()
-        dec = kt[:, 2]
-        sco = kt[:, 0]
-        share = kt.sum(axis=0) / kt.sum()
-        dom = int(np.argmax(share))
-        # the scoring kernel reads the statistics and the S, z, m state (global readout);
-        # the decode kernel reads the union of kept K/V
-        dec_bytes = np.mean([b["kv"] for b in byB])
-        sco_bytes = np.mean([b["stats"] + b["state"] for b in byB])
-        dom_bytes = dec_bytes if dom == 2 else sco_bytes
-        dom_ms = float(np.mean(kt[:, dom]))
-        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-        step_gbs = np.mean([b["total"] for b in by]) / (t_total / K / 1e3) / 1e9
+        sm = summarise(w, m, K, t_max, hbm, peak_kind, world)
         res = {
-            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "metric": METRIC, "value": round(sm["value"], 1), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(t_max / K, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic (seeded, workloads/gen.py)",
@@ -333,30 +388,29 @@ def run_ours(args):
                        "step": "spla_append_kv (1 token/seq) + spla_decode",
                        "l2": "flushed (512 MiB read) before every timed step, outside the events",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-            "roofline": {"bound": "hbm", "kernel": kernel_names[dom],
-                         "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(achieved / hbm, 4),
-                         "traffic": measured_traffic(w.name, int(w.context_lens[0]),
-                                                     kernel_names[dom]),
-                         "peak_kind": f"{peak_kind} hbm_gbs",
-                         "bytes_per_launch": int(dom_bytes), "ms_per_launch": round(dom_ms, 5)},
-            "step_hbm": {"bytes_per_step": int(np.mean([b["total"] for b in by])),
-                         "kv_bytes": int(np.mean([b["kv"] for b in by])),
-                         "stats_bytes": int(np.mean([b["stats"] for b in by])),
-                         "state_bytes": int(np.mean([b["state"] for b in by])),
-                         "achieved_gbs": round(step_gbs, 1),
-                         "frac_of_peak": round(step_gbs / hbm, 4)},
-            "kernels_ms": {n: round(float(np.mean(kt[:, j])), 5) for j, n in enumerate(kernel_names)},
-            "kernel_share": {n: round(float(share[j]), 4) for j, n in enumerate(kernel_names)},
-            "clocks": clk.summary(),
-            # per step: append, length advance, score, select, decode, combine
+            "roofline": sm["roofline"],
+            "step_hbm": sm["step_roofline"],
+            "kernels_ms": sm["kernels_ms"],
+            "kernel_share": sm["kernel_share"],
+            "clocks": m["clocks"],
+            # per step: append, length advance, scoring, selection, decode, combine
             "gpu_launches": 6 * K,
-            "dev_status": status,
+            "dev_status": m["status"],
         }
-        if e2e is not None:
-            res["e2e"] = {"value": round(job_value(world, units_per_step, K, e2e["ms"]), 1),
-                          "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
-                          "d2h_bytes_per_step": e2e["d2h"]}
+        if "e2e" in m:
+            e = m["e2e"]
+            res["e2e"] = {"value": round(job_value(world, w.batch * w.num_q_heads, K, e2e_ms), 1),
+                          "unit": UNIT, "h2d_bytes_per_step": e["h2d"],
+                          "d2h_bytes_per_step": e["d2h"]}
+        if extra:
+            wx, mx, Kx = extra
+            sx = summarise(wx, mx, Kx, tx_max, hbm, peak_kind, world)
+            res[f"also_{wx.name}"] = {
+                "workload": gen.DESCRIPTIONS[wx.name], "steps": Kx,
+                "ms_per_step": round(tx_max / Kx, 5), "value": round(sx["value"], 1),
+                "unit": UNIT, "roofline": sx["roofline"], "step_hbm": sx["step_roofline"],
+                "kernels_ms": sx["kernels_ms"], "dev_status": mx["status"],
+                "clocks": mx["clocks"]}
         if not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(res), flush=True)
@@ -404,11 +458,12 @@ def e2e_pass(w, cache, steps, s0, K, gamma, flush, dev, stream, ones):
 
 # ----------------------------------------------------------------------------- oracle (CPU)
 def _threads():
+    """Threads of the BLAS pool numpy uses (the oracle's only multi-threaded part)."""
     try:
         from threadpoolctl import threadpool_info
         return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
     except Exception:
-        return os.cpu_count() or 1
+        return 1
 
 
 def oracle_sample(w, budget_s: float, steps: int = None):
@@ -437,9 +492,19 @@ def oracle_sample(w, budget_s: float, steps: int = None):
 
 
 def cpu_baseline(w):
-    v, units, secs, desc, n = oracle_sample(w, budget_s=12.0)
-    return {"value": round(v, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
-            "sample": desc}
+    """The oracle on the host cores, twice: BLAS limited to one thread, and at the default
+    pool. numpy runs the oracle's element-wise work on one thread in both; only its matrix
+    products use the pool, so the headline figure states the pool's size, not nproc."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        v1, u1, s1, d1, n1 = oracle_sample(w, budget_s=6.0)
+    vm, um, sm_, dm, nm = oracle_sample(w, budget_s=6.0)
+    return {"value": round(vm, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": dm, "threads_max": {"value": round(vm, 2), "blas_threads": _threads()},
+            "threads_1": {"value": round(v1, 2), "blas_threads": 1, "sample": d1},
+            "nproc": os.cpu_count(),
+            "parallelism": "numpy: matrix products on the BLAS pool, everything else one thread; "
+                           "the oracle decodes one (sequence, KV head) group at a time"}
 
 
 def run_reference(args):
@@ -458,7 +523,9 @@ def run_reference(args):
            "data": "synthetic (seeded, workloads/gen.py)",
            "config": {"workload": gen.DESCRIPTIONS[w.name], "name": w.name},
            "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": _threads(),
-                            "kind": "oracle", "sample": desc},
+                            "kind": "oracle", "sample": desc, "nproc": os.cpu_count(),
+                            "parallelism": "numpy: matrix products on the BLAS pool "
+                                           f"({_threads()} threads), everything else one thread"},
            "e2e": {"value": round(v, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)

@@ -10,9 +10,9 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import (SPLA_BF16, SPLA_F32, SPLA_FLAG_FIRST_ORDER, SPLA_FLAG_NO_RLA, SplaError,
-                   spla_append_kv, spla_cache_init, spla_decode, spla_decode_static_workspace,
-                   spla_decode_workspace_size)
+from ._lib import (SPLA_BF16, SPLA_F32, SPLA_FLAG_FIRST_ORDER, SPLA_FLAG_NO_RLA,
+                   SPLA_WS_STAMP_BYTES, SplaError, spla_append_kv, spla_cache_init, spla_decode,
+                   spla_decode_static_workspace, spla_decode_workspace_size)
 
 __all__ = ["SplaConfig", "SplaDecodeCache", "SplaError", "spla_append_kv", "spla_cache_init",
            "spla_decode", "spla_decode_static_workspace", "spla_decode_workspace_size"]
@@ -81,7 +81,7 @@ class SplaDecodeCache:
                                  self.context_lens.data_ptr(), batch, self.max_blocks_per_seq,
                                  self.num_phys_blocks)
         self.ws_bytes = spla_decode_workspace_size(self.params, batch, self.max_blocks_per_seq)
-        self.workspace = torch.empty((self.ws_bytes + 255) // 256 * 256, dtype=torch.uint8,
+        self.workspace = torch.zeros((self.ws_bytes + 255) // 256 * 256, dtype=torch.uint8,
                                      device=dev)
         self._n_new = torch.zeros((batch,), dtype=torch.int32, device=dev)
         spla_cache_init(self.params, self.c, self._stream(stream))
@@ -141,6 +141,23 @@ class SplaDecodeCache:
                               device=dev)
             orl = torch.empty_like(osp)
         return out, sel, osp, orl
+
+    def scores(self) -> torch.Tensor:
+        """The last decode's block scores, fp32 [batch][Hq][max_blocks_per_seq] (a view of the
+        workspace, whose rows are max_blocks_per_seq rounded up to 4 floats apart; valid after
+        the stream has reached the end of that decode)."""
+        ld = (self.max_blocks_per_seq + 3) // 4 * 4           # rows padded to 16 bytes
+        n = self.batch * self.cfg.num_q_heads * ld
+        off = SPLA_WS_STAMP_BYTES
+        return self.workspace[off:off + 4 * n].view(torch.float32).view(
+            self.batch, self.cfg.num_q_heads, ld)[:, :, :self.max_blocks_per_seq]
+
+    def stamps(self) -> torch.Tensor:
+        """Device timestamps of the last decode's kernels (scoring, selection, decode, combine), a
+        view of the workspace: uint64 [4][256 SM slots][2] = (~ns of the first CTA past its wait, ns
+        of the last CTA's exit), per SM. Zero it (stamps().zero_()) before a call whose times
+        you want; the kernel's span is max(~first) to max(last) over the slots."""
+        return self.workspace[:SPLA_WS_STAMP_BYTES].view(torch.int64).view(4, 256, 2)
 
     def status(self) -> int:
         """Device-detected fault bits (synchronises)."""

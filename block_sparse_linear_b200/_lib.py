@@ -23,6 +23,7 @@ SPLA_DEV_BAD_BLOCK_TABLE = 0x1
 SPLA_DEV_CAPACITY = 0x2
 SPLA_DEV_TIMEOUT = 0x4
 SPLA_DEV_BAD_COUNT = 0x8
+SPLA_DEV_RLA_UNRESOLVED = 0x10
 # dtypes and flags
 SPLA_F32 = 0
 SPLA_BF16 = 1
@@ -30,10 +31,11 @@ SPLA_FLAG_NO_RLA = 0x1
 SPLA_FLAG_FIRST_ORDER = 0x2
 SPLA_MAX_BLOCKS_PER_SEQ = 32768
 SPLA_STATIC_WORKSPACE_BYTES = 16 << 20
+SPLA_WS_STAMP_BYTES = 16384
 
 EXPORTS = ("spla_cache_init", "spla_append_kv", "spla_decode_workspace_size", "spla_decode",
-           "spla_decode_static_workspace", "spla_profile_events", "spla_status_string",
-           "spla_last_cuda_error", "spla_version")
+           "spla_decode_static_workspace", "spla_profile_events", "spla_profile_stamps",
+           "spla_status_string", "spla_last_cuda_error", "spla_version")
 
 
 class spla_params(ctypes.Structure):
@@ -82,8 +84,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.spla_decode.argtypes = [P, C, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     lib.spla_decode_static_workspace.argtypes = [P, C, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.spla_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
+    lib.spla_profile_stamps.argtypes = [i32]
     for f in ("spla_cache_init", "spla_append_kv", "spla_decode_workspace_size", "spla_decode",
-              "spla_decode_static_workspace", "spla_profile_events"):
+              "spla_decode_static_workspace", "spla_profile_events", "spla_profile_stamps"):
         getattr(lib, f).restype = ctypes.c_int
     lib.spla_status_string.argtypes = [ctypes.c_int]
     lib.spla_status_string.restype = ctypes.c_char_p
@@ -134,7 +137,12 @@ def spla_decode_static_workspace(params, cache, q, rms_gamma, out, sel_idx, o_sp
                                                dev_status, stream))
 
 
+def spla_profile_stamps(on: bool):
+    """Turn the kernels' device timestamps (this host thread's decode calls) on or off."""
+    _check("spla_profile_stamps", load().spla_profile_stamps(1 if on else 0))
+
+
 def spla_profile_events(events):
-    """events: five cudaEvent_t handles (ints), or an empty sequence to stop recording."""
+    """events: 2 to 8 cudaEvent_t handles (ints), or an empty sequence to stop recording."""
     arr = (ctypes.c_void_p * max(1, len(events)))(*events)
     _check("spla_profile_events", load().spla_profile_events(arr, len(events)))

@@ -12,12 +12,12 @@ cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s);
 cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, const void* v_new,
                           const int32_t* n_new, int32_t max_new, int32_t* status, cudaStream_t s);
 cudaError_t launch_score(const CacheView& c, const CUtensorMap& tstats, int dtype, const void* q,
-                         double scale, int first_order, float* scores, float* gread,
-                         float* aw, int32_t* status, cudaStream_t s);
+                         double scale, int first_order, float* scores, int ld, float* gread,
+                         float* aw, KernelStamps* stamps, int32_t* status, cudaStream_t s);
 int score_readout_parts(int d);
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
-                          const float* scores, uint32_t* bits, int nw, int32_t* nsel,
-                          int32_t* sel_idx, int kcap, cudaStream_t s);
+                          const float* scores, int ld, uint32_t* bits, int nw, int32_t* nsel,
+                          int32_t* sel_idx, int kcap, KernelStamps* stamps, cudaStream_t s);
 cudaError_t launch_decode_mma(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
                               const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_simt(const CacheView& c, int dtype, const DecodeArgs& a, cudaStream_t s);
@@ -33,11 +33,18 @@ constexpr int kMaxSplit = 512;
 constexpr int kMaxSmem = 227 * 1024;
 
 static thread_local int32_t g_last_cuda_error = 0;
-static thread_local cudaEvent_t g_prof[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
-static thread_local bool g_prof_on = false;
+constexpr int kMaxProfEvents = 8;
+static thread_local cudaEvent_t g_prof[kMaxProfEvents] = {};
+static thread_local int g_prof_n = 0;
+static thread_local bool g_stamps_on = false;
 
+// Event i (0 < i < n) is recorded after the i-th kernel of a decode call, event 0
+// before the first; prof_done() records the ones a shorter chain did not reach.
 static void prof_mark(int i, cudaStream_t s) {
-    if (g_prof_on) cudaEventRecord(g_prof[i], s);
+    if (i < g_prof_n) cudaEventRecord(g_prof[i], s);
+}
+static void prof_done(int next, cudaStream_t s) {
+    for (int i = next; i < g_prof_n; ++i) cudaEventRecord(g_prof[i], s);
 }
 
 void set_last_cuda_error(int32_t e) { g_last_cuda_error = e; }
@@ -95,6 +102,9 @@ static CacheView view_of(const spla_params* p, const spla_cache* c) {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+static_assert((size_t)kStampCount * kStampSlots * sizeof(KernelStamps) <= SPLA_WS_STAMP_BYTES,
+              "timestamp slots fit their region");
+
 static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) {
     DecodeLayout L;
     const int G = p->num_q_heads / p->num_kv_heads;
@@ -103,6 +113,7 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     // a head's bitset row starts on 16 bytes (the decode kernel loads it as int4)
     L.nw = ((mbp + 31) / 32 + 3) & ~3;
     L.rec = rec_floats(p->head_dim);
+    L.ld = (mbp + 3) & ~3;
     const int umax = (int)std::min<int64_t>(mbp, (int64_t)G * L.kcap);
     // one wave: as many splits per group as fit the resident CTA slots, at least 2 blocks each
     int ns = kDecodeSlots / groups;
@@ -110,9 +121,10 @@ static DecodeLayout layout_of(const spla_params* p, int32_t batch, int32_t mbp) 
     L.nsplit = ns;
     L.max_per = (umax + ns - 1) / ns + 1;
     L.readout_parts = score_readout_parts(p->head_dim);
-    size_t off = 0;
+    // the first SPLA_WS_STAMP_BYTES receive the kernels' device timestamps
+    size_t off = SPLA_WS_STAMP_BYTES;
     L.off_scores = off;
-    off = align256(off + (size_t)batch * p->num_q_heads * mbp * sizeof(float));
+    off = align256(off + (size_t)batch * p->num_q_heads * L.ld * sizeof(float));
     L.off_bits = off;
     off = align256(off + (size_t)batch * p->num_q_heads * L.nw * sizeof(uint32_t));
     L.off_nsel = off;
@@ -197,15 +209,19 @@ int32_t spla_last_cuda_error(void) { return g_last_cuda_error; }
 
 spla_status spla_profile_events(void* const* events, int32_t n) {
     if (n == 0) {
-        g_prof_on = false;
+        g_prof_n = 0;
         return SPLA_OK;
     }
-    if (n != 5 || !events) return SPLA_ERR_INVALID_ARG;
-    for (int i = 0; i < 5; ++i) {
+    if (n < 2 || n > kMaxProfEvents || !events) return SPLA_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i)
         if (!events[i]) return SPLA_ERR_INVALID_ARG;
-        g_prof[i] = (cudaEvent_t)events[i];
-    }
-    g_prof_on = true;
+    for (int i = 0; i < n; ++i) g_prof[i] = (cudaEvent_t)events[i];
+    g_prof_n = n;
+    return SPLA_OK;
+}
+
+spla_status spla_profile_stamps(int32_t on) {
+    g_stamps_on = on != 0;
     return SPLA_OK;
 }
 
@@ -259,10 +275,6 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     if (!workspace || workspace_bytes < L.total) return SPLA_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return SPLA_ERR_WORKSPACE;
     const CacheView v = view_of(params, cache);
-    const bool use_mma = params->dtype == SPLA_BF16;
-    const size_t smem = use_mma ? mma_smem_for(v.d, v.bs, L.max_per)
-                                : simt_smem_for(v.d, v.bs, L.max_per);
-    if (smem > (size_t)kMaxSmem) return SPLA_ERR_CAPACITY;
 
     cudaStream_t s = (cudaStream_t)stream;
     char* ws = static_cast<char*>(workspace);
@@ -276,18 +288,24 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     const float eps = params->rms_eps > 0.f ? params->rms_eps : 1e-6f;
     const int first_order = (params->flags & SPLA_FLAG_FIRST_ORDER) ? 1 : 0;
     const int no_rla = (params->flags & SPLA_FLAG_NO_RLA) ? 1 : 0;
+    CUtensorMap tstats;
+    if (!make_stats_map(&tstats, v)) return cuda_fail(cudaErrorInvalidValue);
 
+    // ---- kernel chain: scoring, selection, split-KV decode, combine
+    KernelStamps* stamps = g_stamps_on ? reinterpret_cast<KernelStamps*>(ws) : nullptr;
+    const bool use_mma = params->dtype == SPLA_BF16;
+    const size_t smem = use_mma ? mma_smem_for(v.d, v.bs, L.max_per)
+                                : simt_smem_for(v.d, v.bs, L.max_per);
+    if (smem > (size_t)kMaxSmem) return SPLA_ERR_CAPACITY;
     prof_mark(0, s);
     float* gread = reinterpret_cast<float*>(ws + L.off_gread);
     float* aw_ws = reinterpret_cast<float*>(ws + L.off_aw);
-    CUtensorMap tstats;
-    if (!make_stats_map(&tstats, v)) return cuda_fail(cudaErrorInvalidValue);
-    cudaError_t e = launch_score(v, tstats, params->dtype, q, scale, first_order, scores, gread,
-                                 aw_ws, dev_status, s);
+    cudaError_t e = launch_score(v, tstats, params->dtype, q, scale, first_order, scores, L.ld, gread,
+                                 aw_ws, stamps, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(1, s);
-    e = launch_select(v, params->top_k, params->n_sink, params->n_local, scores, bits, L.nw, nsel,
-                      sel_idx, L.kcap, s);
+    e = launch_select(v, params->top_k, params->n_sink, params->n_local, scores, L.ld, bits, L.nw,
+                      nsel, sel_idx, L.kcap, stamps, s);
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(2, s);
     DecodeArgs da;
@@ -307,6 +325,7 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     da.no_rla = no_rla;
     da.nrd = L.readout_parts;
     da.aw = aw_ws;
+    da.stamps = stamps;
     da.sl2 = sl2;
     da.eps = eps;
     if (use_mma) {
@@ -322,6 +341,7 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     e = launch_combine(v, params->dtype, da, s);
     if (e != cudaSuccess) return cuda_fail(e);
     prof_mark(4, s);
+    prof_done(5, s);
     return SPLA_OK;
 }
 

@@ -39,8 +39,36 @@ struct DecodeLayout {
     int32_t rec;             // floats per partial record
     int32_t readout_parts;   // row ranges of S the global readout is split into
     int32_t max_per;         // union blocks one decode CTA may receive
+    int32_t ld;              // floats between two heads' score rows (mbp rounded up to 4)
     size_t off_scores, off_bits, off_nsel, off_part, off_gread, off_aw, total;
 };
+
+// Device timestamps of one decode call (measurement only), one slot per SM so that
+// CTAs leaving together do not queue on one address: for each kernel of the chain
+// and each SM, ~(first CTA past its dependency wait) and the last CTA's exit, in
+// ns of %globaltimer, raised with atomicMax (so both start from zero). The host
+// takes the extremes over the SMs.
+struct KernelStamps {
+    unsigned long long first_n, last;
+};
+constexpr int kStampSlots = 256;               // >= SMs of the device (148 on a B200)
+enum { kStampScore = 0, kStampSelect = 1, kStampDecode = 2, kStampCombine = 3, kStampCount = 4 };
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ KernelStamps* stamp_slot(KernelStamps* s, int kernel) {
+    uint32_t sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    return s + kernel * kStampSlots + (sm % kStampSlots);
+}
+__device__ __forceinline__ void stamp_first(KernelStamps* s, int kernel) {
+    if (s) atomicMax(&stamp_slot(s, kernel)->first_n, ~global_ns());
+}
+__device__ __forceinline__ void stamp_last(KernelStamps* s, int kernel) {
+    if (s) atomicMax(&stamp_slot(s, kernel)->last, global_ns());
+}
 
 // Per-call arguments of the decode kernels beyond the cache.
 struct DecodeArgs {
@@ -54,6 +82,7 @@ struct DecodeArgs {
     float* part;                // [batch*Hkv][nsplit][G][rec]
     const float* gread;         // [batch*Hkv][nrd][G][d+4]: readout parts, N (d) then D
     const float* aw;            // [batch*Hkv][d][4] phi weights a_g,i (written by the scoring kernel)
+    KernelStamps* stamps;       // [kStampCount][kStampSlots] or null
     int32_t* status;
     int nw, nsplit, max_per, no_rla, nrd;
     float sl2, eps;

@@ -21,7 +21,8 @@
 // combine_kernel (one CTA of 16 warps per query head, launched right behind)
 // merges the head's records: log-sum-exp merge of the softmax partials,
 // o_rla = (N - N~)/(D - D~) with the global readout N, D the scoring kernel
-// computed from S, z; RMSNorm; out = o_sparse + gamma * RMSNorm(o_rla).
+// computed from S, z (the kept blocks' N~, D~ and the subtraction in fp64);
+// RMSNorm; out = o_sparse + gamma * RMSNorm(o_rla).
 //
 // decode_mma_kernel (bf16 K/V): 4 consumer warps + 1 TMA producer warp, three
 // CTAs per SM (128 registers). The pipeline unit is a 64-token tile of one
@@ -335,9 +336,12 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CacheView c, cons
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float* hdr = smem_comb;                     // [ns][4]: m, l, D~
     float* fac = hdr + 4 * ns;                  // [ns]
-    __shared__ __align__(16) float s_po[kCombWarps][D], s_pn[kCombWarps][D];
-    __shared__ float s_M, s_l, s_dt, s_D, s_red[D / 32];
+    __shared__ __align__(16) float s_po[kCombWarps][D];
+    __shared__ __align__(16) double s_pn[kCombWarps][D];
+    __shared__ float s_M, s_l, s_red[D / 32];
+    __shared__ double s_dt, s_D;
     pdl_wait();
+    if (tid == 0) stamp_first(a.stamps, kStampCombine);
     const float* recs = a.part + (((int64_t)b * c.hkv + h) * ns * G + g) * REC;   // split s at s*G*REC
     const float* gr = a.gread + (((int64_t)b * c.hkv + h) * a.nrd * G + g) * (D + 4);
     for (int s = tid; s < ns; s += kCombThreads)
@@ -355,11 +359,11 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CacheView c, cons
             CombVec<D>::load(r + D, ntl[u]);
         }
     }
-    float Nj = 0.f, Dg = 0.f;
+    double Nj = 0.0, Dg = 0.0;
     if (tid < D)
         for (int p = 0; p < a.nrd; ++p) {          // the readout's row-range parts add
-            Nj += __ldcg(gr + (int64_t)p * G * (D + 4) + tid);
-            if (tid == 0) Dg += __ldcg(gr + (int64_t)p * G * (D + 4) + D);
+            Nj += (double)__ldcg(gr + (int64_t)p * G * (D + 4) + tid);
+            if (tid == 0) Dg += (double)__ldcg(gr + (int64_t)p * G * (D + 4) + D);
         }
     if (tid == 0) s_D = Dg;
     const int nsel = a.nsel[(int64_t)b * c.hq + hq];
@@ -371,21 +375,24 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CacheView c, cons
         float M = -SPLA_INF;
         for (int s = lane; s < ns; s += 32) M = fmaxf(M, hdr[4 * s]);
         M = warp_max(M);
-        float l = 0.f, dt = 0.f;
+        float l = 0.f;
+        double dt = 0.0;
         for (int s = lane; s < ns; s += 32) {
             const float f = (M == -SPLA_INF) ? 0.f : ex2(hdr[4 * s] - M);
             fac[s] = f;
             l += hdr[4 * s + 1] * f;
-            dt += hdr[4 * s + 2];
+            dt += (double)hdr[4 * s + 2];
         }
         l = warp_sum(l);
-        dt = warp_sum(dt);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) dt += __shfl_xor_sync(0xffffffffu, dt, o);
         if (lane == 0) { s_M = M; s_l = l; s_dt = dt; }
     }
     __syncthreads();
-    float o[CPL], nt[CPL];
+    float o[CPL];
+    double nt[CPL];
 #pragma unroll
-    for (int e = 0; e < CPL; ++e) o[e] = nt[e] = 0.f;
+    for (int e = 0; e < CPL; ++e) { o[e] = 0.f; nt[e] = 0.0; }
 #pragma unroll
     for (int u = 0; u < kCombPerWarp; ++u) {
         const int s = warp + u * kCombWarps;
@@ -394,7 +401,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CacheView c, cons
 #pragma unroll
             for (int e = 0; e < CPL; ++e) {
                 o[e] = fmaf(acc[u][e], f, o[e]);
-                nt[e] += ntl[u][e];
+                nt[e] += (double)ntl[u][e];
             }
         }
     }
@@ -419,7 +426,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CacheView c, cons
 #pragma unroll
                 for (int e = 0; e < CPL; ++e) {
                     o[e] = fmaf(acc[u][e], f, o[e]);
-                    nt[e] += ntl[u][e];
+                    nt[e] += (double)ntl[u][e];
                 }
             }
         }
@@ -433,16 +440,21 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CacheView c, cons
     // thread j < D finishes column j
     float osp = 0.f, orl = 0.f;
     if (tid < D) {
-        float ot = 0.f, ntt = 0.f;
+        float ot = 0.f;
+        double ntt = 0.0;
 #pragma unroll
         for (int w = 0; w < kCombWarps; ++w) {
             ot += s_po[w][tid];
             ntt += s_pn[w][tid];
         }
-        const float lsum = s_l, Dr = s_D - s_dt;
-        const bool off = a.no_rla || nsel >= nb || !(Dr > 0.f) || L == 0;
+        const float lsum = s_l;
+        const double Dr = s_D - s_dt;
+        const bool off = a.no_rla || nsel >= nb || L == 0;
+        // the residual mass is below what the state resolves: o_rla = 0, and the caller is told
+        const bool unresolved = !off && !(Dr > 0.0);
+        if (unresolved && tid == 0) set_status(a.status, SPLA_DEV_RLA_UNRESOLVED);
         osp = (lsum > 0.f) ? ot / lsum : 0.f;
-        orl = off ? 0.f : (Nj - ntt) / Dr;
+        orl = (off || unresolved) ? 0.f : (float)((Nj - ntt) / Dr);
         // RMS of o_rla over the head dimension
         const float sq = warp_sum(orl * orl);
         if (lane == 0) s_red[warp] = sq;
@@ -459,6 +471,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CacheView c, cons
         if (a.o_sp) a.o_sp[oi] = osp;
         if (a.o_rl) a.o_rl[oi] = orl;
     }
+    if (tid == 0) stamp_last(a.stamps, kStampCombine);
 }
 
 // ------------------------------------------------------------------ bf16 tensor-core kernel
@@ -475,8 +488,8 @@ struct MmaCfg {
 
 template <int D, int UPB, int STAGES>
 __global__ void __launch_bounds__(MmaCfg<D, UPB, STAGES>::THREADS, 3)
-decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const DecodeArgs a) {
+decode_mma_kernel(const __grid_constant__ CacheView c, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ DecodeArgs a) {
     using Cfg = MmaCfg<D, UPB, STAGES>;
     constexpr int NCW = Cfg::NCW, G4 = 4, BS = Cfg::BS;
     extern __shared__ __align__(1024) unsigned char smem_mma[];
@@ -559,6 +572,7 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         }
     }
     pdl_wait();
+    if (tid == 0) stamp_first(a.stamps, kStampDecode);
     // the group's selections (one round of loads by every thread), then every
     // thread builds its words' part of this CTA's share of their union
     if (nb > 0) {
@@ -579,6 +593,7 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
             const int g = e / REC, f = e % REC;
             a.part[(rec_base + g) * REC + f] = (f == 0) ? -SPLA_INF : 0.f;
         }
+        if (tid == 0) stamp_last(a.stamps, kStampDecode);
         return;
     }
 
@@ -818,13 +833,15 @@ decode_mma_kernel(CacheView c, const __grid_constant__ CUtensorMap tmK,
         *reinterpret_cast<float4*>(rec + 4 + D + j) = nt;
         if (j == 0) *reinterpret_cast<float4*>(rec) = make_float4(M, l, dt, 0.f);
     }
+    if (tid == 0) stamp_last(a.stamps, kStampDecode);
 }
 
 // ------------------------------------------------------------------ fp32 SIMT kernel
 // One CTA of 256 threads per (split, group). Tiles are staged through shared
 // memory as fp32; every product and sum is an fp32 FMA.
 template <typename T>
-__global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const DecodeArgs a) {
+__global__ void __launch_bounds__(256) decode_simt_kernel(const __grid_constant__ CacheView c,
+                                                          const __grid_constant__ DecodeArgs a) {
     extern __shared__ __align__(16) unsigned char smem_simt[];
     const int d = c.d, BS = c.bs, G = c.group;
     float* Ks = reinterpret_cast<float*>(smem_simt);       // [BS][d]
@@ -864,6 +881,7 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const Dec
     stage_query(a.q, a.aw, c.m, c.table, c.mbp, c.hq, c.hkv, G, d, sizeof(T) == 2, b, h, qs, ml,
                 aw, nullptr, tid, blockDim.x);
     pdl_wait();
+    if (tid == 0) stamp_first(a.stamps, kStampDecode);
     stage_bits(a.bits, a.nw, c.hq, G, b, h, nwu, wbits, tid, blockDim.x);
     __syncthreads();
     const int nblk = union_share(c.table + (int64_t)b * c.mbp, c.num_phys, G, wbits, nwu, nb,
@@ -965,6 +983,7 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(CacheView c, const Dec
             }
         }
     }
+    if (tid == 0) stamp_last(a.stamps, kStampDecode);
 }
 
 // ------------------------------------------------------------------ host launchers

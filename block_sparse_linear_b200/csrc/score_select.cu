@@ -111,8 +111,9 @@ template <> struct QVec<float> {
 template <int D, typename T>
 __global__ void __launch_bounds__(kScoreWarps * 32, kScoreCtasPerSm)
 score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* __restrict__ q,
-             double scale, double log_bs, int first_order, float* __restrict__ scores,
-             float* __restrict__ gread, float* __restrict__ aw_out, int ntile, int32_t* status) {
+             double scale, double log_bs, int first_order, float* __restrict__ scores, int ld,
+             float* __restrict__ gread, float* __restrict__ aw_out, int ntile, KernelStamps* stamps,
+             int32_t* status) {
     using S = ScoreShape<D>;
     constexpr int RP = S::kReadoutParts, TS = S::kTileStages, RPS = S::kRowsPerStage;
     constexpr int CPL = D / 32;                    // rows per lane in the readout weights
@@ -164,6 +165,7 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
         fence_barrier_init();
     }
     pdl_wait();          // statistics, state and lengths come from the append kernels
+    if (threadIdx.x == 0) stamp_first(stamps, kStampScore);
     for (int b = threadIdx.x; b < min(c.batch, kScoreNbSmem); b += blockDim.x) {
         const int32_t L = c.lens[b];
         if (blockIdx.x == 0 && (L < 0 || L > mbp * bs)) set_status(status, SPLA_DEV_CAPACITY);
@@ -458,12 +460,14 @@ score_kernel(const __grid_constant__ CUtensorMap tstats, CacheView c, const T* _
                             // while the argument stays below e^4 - 1
                             sc += (double)log1pf((float)(0.5 * (e ? oth1 : oth0)));
                         }
-                        scores[((int64_t)b * c.hq + h * G + g) * mbp + j] = (float)sc;
+                        scores[((int64_t)b * c.hq + h * G + g) * ld + j] = (float)sc;
                     }
                 }
             }
         }
     }
+    // (a warp that left early on a failed wait stamps nothing: the status says it failed)
+    if (threadIdx.x == 0) stamp_last(stamps, kStampScore);
 }
 
 // ------------------------------------------------------------------ selection
@@ -550,9 +554,10 @@ __device__ __forceinline__ void rank_candidates(uint32_t* keys, const uint32_t* 
 // carries a dependency through shared memory.
 template <int NT>
 __global__ void __launch_bounds__(NT) select_kernel(CacheView c, int top_k, int n_sink,
-                                                    int n_local, const float* scores,
+                                                    int n_local, const float* scores, int ld,
                                                     uint32_t* bits, int nw, int32_t* nsel,
-                                                    int32_t* sel_idx, int kcap) {
+                                                    int32_t* sel_idx, int kcap,
+                                                    KernelStamps* stamps) {
     constexpr int kSelThreads = NT;
     constexpr int kSelWarps = NT / 32;
     constexpr int kWordsPerThread = SPLA_MAX_BLOCKS_PER_SEQ / 32 / NT;
@@ -579,7 +584,8 @@ __global__ void __launch_bounds__(NT) select_kernel(CacheView c, int top_k, int 
     // the decode kernels launch only now: before their own wait they may read what
     // the scoring kernel wrote (it has completed)
     pdl_trigger();
-    const float* sc = scores + ((int64_t)b * c.hq + hq) * c.mbp;
+    if (tid == 0) stamp_first(stamps, kStampSelect);
+    const float* sc = scores + ((int64_t)b * c.hq + hq) * ld;
     // the first batch of score loads goes out with the length load, bounded by the
     // capacity (entries past the sequence's blocks are loaded and ignored)
     constexpr int kKeyBatch = 8;
@@ -887,13 +893,16 @@ __global__ void __launch_bounds__(NT) select_kernel(CacheView c, int top_k, int 
         }
         for (int i = total + tid; i < kcap; i += kSelThreads) out[i] = -1;
     }
-    if (tid == 0) nsel[(int64_t)b * c.hq + hq] = total;
+    if (tid == 0) {
+        nsel[(int64_t)b * c.hq + hq] = total;
+        stamp_last(stamps, kStampSelect);
+    }
 }
 
 template <int D, typename T>
 static cudaError_t launch_score_t(const CacheView& c, const CUtensorMap& tstats, const void* q,
-                                  double scale, int first_order, float* scores, float* gread,
-                                  float* aw, int32_t* status, cudaStream_t s) {
+                                  double scale, int first_order, float* scores, int ld, float* gread,
+                                  float* aw, KernelStamps* stamps, int32_t* status, cudaStream_t s) {
     using S = ScoreShape<D>;
     const int groups = c.batch * c.hkv;
     const int ntile = (c.mbp + kTile - 1) / kTile;
@@ -906,8 +915,8 @@ static cudaError_t launch_score_t(const CacheView& c, const CUtensorMap& tstats,
     e = cudaFuncSetAttribute(score_kernel<D, T>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     return launch_pdl(score_kernel<D, T>, dim3(grid), dim3(kScoreWarps * 32), S::kSmem, s, tstats,
-                      c, (const T*)q, scale, log((double)c.bs), first_order, scores, gread, aw,
-                      ntile, status);
+                      c, (const T*)q, scale, log((double)c.bs), first_order, scores, ld, gread, aw,
+                      ntile, stamps, status);
 }
 
 int score_readout_parts(int d) {
@@ -915,18 +924,18 @@ int score_readout_parts(int d) {
 }
 
 cudaError_t launch_score(const CacheView& c, const CUtensorMap& tstats, int dtype, const void* q,
-                         double scale, int first_order, float* scores, float* gread,
-                         float* aw, int32_t* status, cudaStream_t s) {
+                         double scale, int first_order, float* scores, int ld, float* gread,
+                         float* aw, KernelStamps* stamps, int32_t* status, cudaStream_t s) {
     if (dtype == SPLA_BF16)
-        return c.d == 128 ? launch_score_t<128, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, gread, aw, status, s)
-                          : launch_score_t<64, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, gread, aw, status, s);
-    return c.d == 128 ? launch_score_t<128, float>(c, tstats, q, scale, first_order, scores, gread, aw, status, s)
-                      : launch_score_t<64, float>(c, tstats, q, scale, first_order, scores, gread, aw, status, s);
+        return c.d == 128 ? launch_score_t<128, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, ld, gread, aw, stamps, status, s)
+                          : launch_score_t<64, __nv_bfloat16>(c, tstats, q, scale, first_order, scores, ld, gread, aw, stamps, status, s);
+    return c.d == 128 ? launch_score_t<128, float>(c, tstats, q, scale, first_order, scores, ld, gread, aw, stamps, status, s)
+                      : launch_score_t<64, float>(c, tstats, q, scale, first_order, scores, ld, gread, aw, stamps, status, s);
 }
 
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
-                          const float* scores, uint32_t* bits, int nw, int32_t* nsel,
-                          int32_t* sel_idx, int kcap, cudaStream_t s) {
+                          const float* scores, int ld, uint32_t* bits, int nw, int32_t* nsel,
+                          int32_t* sel_idx, int kcap, KernelStamps* stamps, cudaStream_t s) {
     const size_t smem = (size_t)((c.mbp + 31) / 32) * 32 * sizeof(uint32_t);
     const bool lng = c.mbp > kSelLongBlocks;
     auto kern = lng ? select_kernel<kSelThreadsLong> : select_kernel<512>;
@@ -934,7 +943,7 @@ cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(c.batch * c.hq), dim3(lng ? kSelThreadsLong : 512), smem, s, c,
-                      top_k, n_sink, n_local, scores, bits, nw, nsel, sel_idx, kcap);
+                      top_k, n_sink, n_local, scores, ld, bits, nw, nsel, sel_idx, kcap, stamps);
 }
 
 }  // namespace spla

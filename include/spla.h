@@ -64,6 +64,8 @@ typedef enum {
 #define SPLA_DEV_CAPACITY        0x2   /* a length or an append past max_blocks_per_seq*B */
 #define SPLA_DEV_TIMEOUT         0x4   /* a bounded wait on a TMA barrier ran out */
 #define SPLA_DEV_BAD_COUNT       0x8   /* n_new[b] outside [0, max_new] */
+#define SPLA_DEV_RLA_UNRESOLVED  0x10  /* a head's residual denominator D - D~ was not positive:
+                                          its o_rla was set to 0 (see spla_decode) */
 
 typedef enum { SPLA_F32 = 0, SPLA_BF16 = 1 } spla_dtype;
 
@@ -145,6 +147,22 @@ SPLA_API spla_status spla_append_kv(const spla_params* params, const spla_cache*
                            int32_t max_new, int32_t* dev_status, void* stream);
 
 /*
+ * Layout facts of the decode workspace that callers may rely on (measurement and
+ * tests; the rest of the workspace is private):
+ *   bytes [0, SPLA_WS_STAMP_BYTES): device timestamps of the last call's kernels
+ *     (written only while spla_profile_stamps is on for the calling thread),
+ *     uint64 [4 kernels: scoring, selection, decode, combine][256 SM slots][2]: per SM, ~t
+ *     of the first CTA past its dependency wait and t of the last CTA's exit, ns of
+ *     %globaltimer, raised with atomicMax (the kernel's span is the maximum of the
+ *     first entries, complemented, to the maximum of the second). A caller that
+ *     reads them zeroes these bytes before the call; nothing else depends on them.
+ *   from byte SPLA_WS_STAMP_BYTES: the last call's block scores (log of the Taylor
+ *     estimate), fp32 [batch][Hq][ld], ld = max_blocks_per_seq rounded up to a
+ *     multiple of 4; entries past a sequence's blocks are undefined.
+ */
+#define SPLA_WS_STAMP_BYTES 16384u
+
+/*
  * Bytes of scratch spla_decode needs for this shape (host-only, no CUDA call).
  * The value depends only on its arguments.
  */
@@ -161,12 +179,16 @@ SPLA_API spla_status spla_decode_workspace_size(const spla_params* params, int32
  *   o_sparse_dbg, o_rla_dbg : [batch][Hq][d] fp32 or NULL: the two branches
  *                before the combine.
  *   workspace  : device scratch of >= spla_decode_workspace_size bytes,
- *                256-byte aligned; its contents need no initialisation.
+ *                256-byte aligned; its contents need no initialisation. Calls
+ *                that share a workspace must be ordered on the GPU (one stream,
+ *                or events).
  *   dev_status : int32 (device) or NULL.
  * Decode attends over tokens [0, context_lens[b]). An empty sequence gives
- * out = 0. o_rla is 0 when every block is kept, or when the residual
- * denominator D - D~ is not positive in fp32 (the residual mass is below the
- * state's resolution). Selection ties go to the lower block index.
+ * out = 0. o_rla is 0 when every block is kept. When the residual denominator
+ * D - D~ (the linear-attention mass of the blocks not kept, by subtraction) is
+ * not positive in the arithmetic of the kernels, the unkept mass is below the
+ * state's resolution: that head's o_rla is set to 0 and SPLA_DEV_RLA_UNRESOLVED
+ * is OR-ed into *dev_status. Selection ties go to the lower block index.
  */
 SPLA_API spla_status spla_decode(const spla_params* params, const spla_cache* cache, const void* q,
                         const float* rms_gamma, void* out, int32_t* sel_idx,
@@ -209,14 +231,23 @@ SPLA_API spla_status spla_decode_static_workspace(const spla_params* params,
                                          int32_t* dev_status, void* stream);
 
 /*
- * Measurement hook (no part of the method). With n == 5, every later
- * spla_decode call made from this host thread records events[0..4]
- * (cudaEvent_t handles) on its stream: before the scoring kernel, after it,
- * after the selection kernel, after the split-KV decode kernel and after the
- * combine kernel. n == 0 turns it off. The handles are copied; the events stay
- * the caller's. Returns SPLA_ERR_INVALID_ARG for any other n or a NULL array.
+ * Measurement hook (no part of the method). With 2 <= n <= 8, every later
+ * spla_decode call made from this host thread records events[0..n-1]
+ * (cudaEvent_t handles) on its stream: events[0] before its first kernel and
+ * events[i] after its i-th kernel; events past the call's last kernel are
+ * recorded right after it. spla_decode runs four kernels: scoring, selection,
+ * split-KV decode and combine. n == 0 turns it off. The handles are copied; the events stay the caller's. Returns
+ * SPLA_ERR_INVALID_ARG for any other n or a NULL array or handle.
  */
 SPLA_API spla_status spla_profile_events(void* const* events, int32_t n);
+
+/*
+ * Measurement hook (no part of the method). With on != 0, later spla_decode calls
+ * made from this host thread write their kernels' device timestamps into the
+ * first SPLA_WS_STAMP_BYTES of the workspace (see SPLA_WS_STAMP_BYTES); with
+ * on == 0 (the default) the kernels skip them.
+ */
+SPLA_API spla_status spla_profile_stamps(int32_t on);
 
 /* Human-readable name of a status (static storage). */
 SPLA_API const char* spla_status_string(spla_status s);
