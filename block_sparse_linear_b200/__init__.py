@@ -2,7 +2,8 @@
 
 ``SplaDecodeCache`` holds the device buffers of include/spla.h's ``spla_cache``
 (allocated with PyTorch, which is used for device memory and streams only) and
-forwards ``append`` / ``decode`` to ``spla_append_kv`` / ``spla_decode``. Every
+forwards ``append`` / ``decode`` to ``spla_append_kv`` (or ``spla_append_kv_bulk``
+for long chunks) / ``spla_decode``. Every
 step of the decode path runs in the library's kernels; there is no fallback.
 """
 from dataclasses import dataclass
@@ -11,11 +12,16 @@ import torch
 
 from . import _lib
 from ._lib import (SPLA_BF16, SPLA_F32, SPLA_FLAG_FIRST_ORDER, SPLA_FLAG_NO_RLA,
-                   SPLA_WS_STAMP_BYTES, SplaError, spla_append_kv, spla_cache_init, spla_decode,
-                   spla_decode_static_workspace, spla_decode_workspace_size)
+                   SPLA_WS_STAMP_BYTES, SplaError, spla_append_bulk_workspace_size, spla_append_kv,
+                   spla_append_kv_bulk, spla_cache_init, spla_decode, spla_decode_static_workspace,
+                   spla_decode_workspace_size)
 
-__all__ = ["SplaConfig", "SplaDecodeCache", "SplaError", "spla_append_kv", "spla_cache_init",
-           "spla_decode", "spla_decode_static_workspace", "spla_decode_workspace_size"]
+__all__ = ["SplaConfig", "SplaDecodeCache", "SplaError", "spla_append_bulk_workspace_size",
+           "spla_append_kv", "spla_append_kv_bulk", "spla_cache_init", "spla_decode",
+           "spla_decode_static_workspace", "spla_decode_workspace_size"]
+
+# Chunks at least this long go through spla_append_kv_bulk where it applies.
+BULK_MIN_TOKENS = 64
 
 
 @dataclass
@@ -84,21 +90,40 @@ class SplaDecodeCache:
         self.workspace = torch.zeros((self.ws_bytes + 255) // 256 * 256, dtype=torch.uint8,
                                      device=dev)
         self._n_new = torch.zeros((batch,), dtype=torch.int32, device=dev)
+        self._bulk_ws = None
         spla_cache_init(self.params, self.c, self._stream(stream))
 
     def _stream(self, stream=None) -> int:
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         return s.cuda_stream
 
+    def bulk_supported(self) -> bool:
+        """Whether spla_append_kv_bulk takes this cache's shape (bf16, head_dim 128)."""
+        return self.cfg.dtype == "bf16" and self.cfg.head_dim == 128
+
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, n_new: torch.Tensor = None,
-               stream=None) -> None:
-        """k_new, v_new: [batch][max_new][Hkv][d] on the device; n_new: [batch] int32 (device)."""
+               stream=None, bulk: bool = None) -> None:
+        """k_new, v_new: [batch][max_new][Hkv][d] on the device; n_new: [batch] int32 (device).
+        bulk: None picks spla_append_kv_bulk for chunks of BULK_MIN_TOKENS or more where the
+        shape allows it; True asks for it (SplaError if unsupported); False never uses it."""
         assert k_new.is_contiguous() and v_new.is_contiguous()
         assert k_new.dtype == self.cfg.torch_dtype and v_new.dtype == self.cfg.torch_dtype
         max_new = int(k_new.shape[1])
         if n_new is None:
             self._n_new.fill_(max_new)
             n_new = self._n_new
+        if bulk is None:
+            bulk = self.bulk_supported() and max_new >= BULK_MIN_TOKENS
+        if bulk:
+            need = spla_append_bulk_workspace_size(self.params, self.batch, max_new)
+            if self._bulk_ws is None or self._bulk_ws.numel() < need:
+                self._bulk_ws = torch.empty((max(need, 16) + 255) // 256 * 256,
+                                            dtype=torch.uint8, device=self.device)
+            spla_append_kv_bulk(self.params, self.c, k_new.data_ptr(), v_new.data_ptr(),
+                                n_new.data_ptr(), max_new, self._bulk_ws.data_ptr(),
+                                self._bulk_ws.numel(), self.dev_status.data_ptr(),
+                                self._stream(stream))
+            return
         spla_append_kv(self.params, self.c, k_new.data_ptr(), v_new.data_ptr(), n_new.data_ptr(),
                        max_new, self.dev_status.data_ptr(), self._stream(stream))
 

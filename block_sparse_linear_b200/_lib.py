@@ -33,7 +33,8 @@ SPLA_MAX_BLOCKS_PER_SEQ = 32768
 SPLA_STATIC_WORKSPACE_BYTES = 16 << 20
 SPLA_WS_STAMP_BYTES = 16384
 
-EXPORTS = ("spla_cache_init", "spla_append_kv", "spla_decode_workspace_size", "spla_decode",
+EXPORTS = ("spla_cache_init", "spla_append_kv", "spla_append_kv_bulk",
+           "spla_append_bulk_workspace_size", "spla_decode_workspace_size", "spla_decode",
            "spla_decode_static_workspace", "spla_profile_events", "spla_profile_stamps",
            "spla_status_string", "spla_last_cuda_error", "spla_version")
 
@@ -80,6 +81,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                          ctypes.c_int32, ctypes.c_size_t)
     lib.spla_cache_init.argtypes = [P, C, vp]
     lib.spla_append_kv.argtypes = [P, C, vp, vp, vp, i32, vp, vp]
+    lib.spla_append_kv_bulk.argtypes = [P, C, vp, vp, vp, i32, vp, sz, vp, vp]
+    lib.spla_append_bulk_workspace_size.argtypes = [P, i32, i32, ctypes.POINTER(sz)]
     lib.spla_decode_workspace_size.argtypes = [P, i32, i32, ctypes.POINTER(sz)]
     lib.spla_decode.argtypes = [P, C, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     lib.spla_decode_static_workspace.argtypes = [P, C, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -111,6 +114,22 @@ def spla_append_kv(params, cache, k_new, v_new, n_new, max_new, dev_status, stre
     _check("spla_append_kv", load().spla_append_kv(ctypes.byref(params), ctypes.byref(cache),
                                                    k_new, v_new, n_new, max_new, dev_status,
                                                    stream))
+
+
+def spla_append_kv_bulk(params, cache, k_new, v_new, n_new, max_new, workspace, workspace_bytes,
+                        dev_status, stream=0):
+    _check("spla_append_kv_bulk",
+           load().spla_append_kv_bulk(ctypes.byref(params), ctypes.byref(cache), k_new, v_new,
+                                      n_new, max_new, workspace, workspace_bytes, dev_status,
+                                      stream))
+
+
+def spla_append_bulk_workspace_size(params, batch, max_new) -> int:
+    n = ctypes.c_size_t(0)
+    _check("spla_append_bulk_workspace_size",
+           load().spla_append_bulk_workspace_size(ctypes.byref(params), batch, max_new,
+                                                  ctypes.byref(n)))
+    return n.value
 
 
 def spla_decode_workspace_size(params, batch, max_blocks_per_seq) -> int:

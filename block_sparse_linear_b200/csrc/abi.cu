@@ -11,6 +11,10 @@ namespace spla {
 cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s);
 cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, const void* v_new,
                           const int32_t* n_new, int32_t max_new, int32_t* status, cudaStream_t s);
+cudaError_t launch_append_bulk(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const void* k_new, const void* v_new, const int32_t* n_new,
+                               int32_t max_new, float* part, int32_t* status, cudaStream_t s);
+size_t bulk_workspace_bytes(int batch, int hkv, int d, int max_new);
 cudaError_t launch_score(const CacheView& c, const CUtensorMap& tstats, int dtype, const void* q,
                          double scale, int first_order, float* scores, int ld, float* gread,
                          float* aw, KernelStamps* stamps, int32_t* status, cudaStream_t s);
@@ -185,6 +189,21 @@ static bool make_stats_map(CUtensorMap* m, const CacheView& c) {
     return r == CUDA_SUCCESS;
 }
 
+// 3-D view of an append input [batch*max_new rows][Hkv][d] bf16; box = 64 dims x 1 head
+// x 64 tokens (8 KiB), 128B swizzle; rows past the end read as zero.
+static bool make_input_map(CUtensorMap* m, const void* x, const CacheView& c, int32_t max_new) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)c.d, (cuuint64_t)c.hkv, (cuuint64_t)c.batch * max_new};
+    cuuint64_t strides[2] = {(cuuint64_t)c.d * 2, (cuuint64_t)c.hkv * c.d * 2};
+    cuuint32_t box[3] = {64u, 1u, 64u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace spla
 
 using namespace spla;
@@ -245,6 +264,56 @@ spla_status spla_append_kv(const spla_params* params, const spla_cache* cache, c
     const CacheView v = view_of(params, cache);
     cudaError_t e = launch_append(v, params->dtype, k_new, v_new, n_new, max_new, dev_status,
                                   (cudaStream_t)stream);
+    return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
+}
+
+static spla_status check_bulk(const spla_params* params, int32_t batch, int32_t max_new) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if (params->dtype != SPLA_BF16 || params->head_dim != 128) return SPLA_ERR_UNSUPPORTED;
+    if (batch <= 0 || max_new < 0) return SPLA_ERR_INVALID_ARG;
+    if ((int64_t)batch * max_new > INT32_MAX) return SPLA_ERR_CAPACITY;
+    return SPLA_OK;
+}
+
+spla_status spla_append_bulk_workspace_size(const spla_params* params, int32_t batch,
+                                            int32_t max_new, size_t* bytes) {
+    spla_status st = check_bulk(params, batch, max_new);
+    if (st != SPLA_OK) return st;
+    if (!bytes) return SPLA_ERR_INVALID_ARG;
+    *bytes = max_new > 0 ? bulk_workspace_bytes(batch, params->num_kv_heads, params->head_dim,
+                                                max_new)
+                         : 0;
+    return SPLA_OK;
+}
+
+spla_status spla_append_kv_bulk(const spla_params* params, const spla_cache* cache,
+                                const void* k_new, const void* v_new, const int32_t* n_new,
+                                int32_t max_new, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, void* stream) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if ((st = check_cache(cache)) != SPLA_OK) return st;
+    if ((st = check_bulk(params, cache->batch, max_new)) != SPLA_OK) return st;
+    if (!n_new) return SPLA_ERR_INVALID_ARG;
+    const CacheView v = view_of(params, cache);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (max_new == 0) {
+        cudaError_t e = launch_append(v, params->dtype, k_new, v_new, n_new, 0, dev_status, s);
+        return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
+    }
+    if (!k_new || !v_new || (reinterpret_cast<uintptr_t>(k_new) & 15) ||
+        (reinterpret_cast<uintptr_t>(v_new) & 15))
+        return SPLA_ERR_INVALID_ARG;
+    const size_t need = bulk_workspace_bytes(cache->batch, params->num_kv_heads, params->head_dim,
+                                             max_new);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15))
+        return SPLA_ERR_WORKSPACE;
+    CUtensorMap tk, tv;
+    if (!make_input_map(&tk, k_new, v, max_new) || !make_input_map(&tv, v_new, v, max_new))
+        return SPLA_ERR_UNSUPPORTED;
+    cudaError_t e = launch_append_bulk(v, tk, tv, k_new, v_new, n_new, max_new,
+                                       reinterpret_cast<float*>(workspace), dev_status, s);
     return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
 }
 

@@ -236,30 +236,42 @@ cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// The block role alone: tokens into the pool and the touched blocks' statistics.
+cudaError_t launch_append_blocks(const CacheView& c, int dtype, const void* k_new,
+                                 const void* v_new, const int32_t* n_new, int32_t max_new,
+                                 int32_t* status, cudaStream_t s, bool with_rows) {
+    const int nsb = (max_new + c.bs - 1) / c.bs + 1;         // blocks a sequence's tokens can touch
+    dim3 grid(nsb + (with_rows ? (c.d + 7) / 8 : 0), c.batch * c.hkv);
+    const size_t smem = (size_t)c.bs * c.d * sizeof(float);
+    cudaError_t e = dtype == SPLA_BF16
+        ? cudaFuncSetAttribute(append_kernel<__nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+        : cudaFuncSetAttribute(append_kernel<float>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (dtype == SPLA_BF16) {
+        using B16 = __nv_bfloat16;
+        return launch_pdl(append_kernel<B16>, grid, dim3(256), smem, s, c, (const B16*)k_new,
+                          (const B16*)v_new, n_new, max_new, nsb, status);
+    }
+    return launch_pdl(append_kernel<float>, grid, dim3(256), smem, s, c, (const float*)k_new,
+                      (const float*)v_new, n_new, max_new, nsb, status);
+}
+
+cudaError_t launch_append_advance(const CacheView& c, const int32_t* n_new, int32_t max_new,
+                                  cudaStream_t s) {
+    return launch_pdl(append_advance_kernel, dim3(1), dim3(128), 0, s, c, n_new, max_new);
+}
+
 cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, const void* v_new,
                           const int32_t* n_new, int32_t max_new, int32_t* status,
                           cudaStream_t s) {
     if (max_new > 0) {
-        const int nsb = (max_new + c.bs - 1) / c.bs + 1;     // blocks a sequence's tokens can touch
-        dim3 grid(nsb + (c.d + 7) / 8, c.batch * c.hkv);
-        const size_t smem = (size_t)c.bs * c.d * sizeof(float);
-        cudaError_t e = dtype == SPLA_BF16
-            ? cudaFuncSetAttribute(append_kernel<__nv_bfloat16>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-            : cudaFuncSetAttribute(append_kernel<float>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        if (dtype == SPLA_BF16) {
-            using B16 = __nv_bfloat16;
-            e = launch_pdl(append_kernel<B16>, grid, dim3(256), smem, s, c, (const B16*)k_new,
-                           (const B16*)v_new, n_new, max_new, nsb, status);
-        } else {
-            e = launch_pdl(append_kernel<float>, grid, dim3(256), smem, s, c, (const float*)k_new,
-                           (const float*)v_new, n_new, max_new, nsb, status);
-        }
+        cudaError_t e = launch_append_blocks(c, dtype, k_new, v_new, n_new, max_new, status, s,
+                                             /*with_rows=*/true);
         if (e != cudaSuccess) return e;
     }
-    return launch_pdl(append_advance_kernel, dim3(1), dim3(128), 0, s, c, n_new, max_new);
+    return launch_append_advance(c, n_new, max_new, s);
 }
 
 }  // namespace spla

@@ -147,6 +147,35 @@ SPLA_API spla_status spla_append_kv(const spla_params* params, const spla_cache*
                            int32_t max_new, int32_t* dev_status, void* stream);
 
 /*
+ * a0 for many tokens per call (a prefill, or a long chunk) -- the same result as
+ * spla_append_kv up to fp32 rounding order, with the global state's sum over the
+ * new tokens, phi(K)^T V, run as a dense contraction on the tensor cores (section
+ * 2.2: the state accumulates phi(k) v^T over every token; section 2.3: phi = exp).
+ * Arguments as for spla_append_kv, plus:
+ *   workspace       : device scratch of at least spla_append_bulk_workspace_size
+ *                     bytes, 16-byte aligned, owned by the caller; the call reads
+ *                     and writes it on `stream` only, so calls on one stream may
+ *                     share it. Its contents need no initialisation.
+ * Supported: params->dtype == SPLA_BF16 and head_dim == 128 (SPLA_ERR_UNSUPPORTED
+ * otherwise; spla_append_kv covers every shape); k_new and v_new 16-byte aligned
+ * (SPLA_ERR_INVALID_ARG otherwise). The new tokens of a sequence are cut into
+ * splits of whole 64-token tiles; every split's partial state (S_c, z_c at its
+ * own maximum m_c) is merged into S, z, m in split order, so repeated calls give
+ * bit-identical results. Device faults as for spla_append_kv.
+ */
+SPLA_API spla_status spla_append_kv_bulk(const spla_params* params, const spla_cache* cache,
+                                const void* k_new, const void* v_new, const int32_t* n_new,
+                                int32_t max_new, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, void* stream);
+
+/*
+ * Bytes of scratch spla_append_kv_bulk needs for (batch, max_new) under params
+ * (host-only, no CUDA call; depends only on its arguments).
+ */
+SPLA_API spla_status spla_append_bulk_workspace_size(const spla_params* params, int32_t batch,
+                                            int32_t max_new, size_t* bytes);
+
+/*
  * Layout facts of the decode workspace that callers may rely on (measurement and
  * tests; the rest of the workspace is private):
  *   bytes [0, SPLA_WS_STAMP_BYTES): device timestamps of the last call's kernels
