@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the bulk-append (prefill chunk) measurement")
     ap.add_argument("--also", default="cfg4",
                     help="a second workload measured in the same run ('' for none)")
     return ap.parse_args()
@@ -368,6 +370,8 @@ def run_ours(args):
         mx = measure(wx, Kx, W, dev, stream, flush, rank_sync, with_e2e=False)
         extra = (wx, mx, Kx)
 
+    prefill = measure_prefill("cfg4", dev, stream, flush) if not args.no_prefill else None
+
     # ---- max over ranks (the same single collective on every rank)
     t_max, e2e_ms, tx_max = max_over_ranks(
         [t_total, m["e2e"]["ms"] if "e2e" in m else 0.0,
@@ -411,12 +415,66 @@ def run_ours(args):
                 "unit": UNIT, "roofline": sx["roofline"], "step_hbm": sx["step_roofline"],
                 "kernels_ms": sx["kernels_ms"], "dev_status": mx["status"],
                 "clocks": mx["clocks"]}
+        if prefill:
+            hbm_p = hbm
+            prefill["bulk"]["frac_of_measured_peak" if peak_kind == "measured"
+                            else "frac_of_fallback_peak"] = round(
+                prefill["bulk"]["achieved_gbs"] / hbm_p, 4)
+            res["bulk_append"] = prefill
         if not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(res), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_prefill(name, dev, stream, flush, n_tok=8192, K=8, W=2):
+    """Bulk append of one n_tok-token chunk per sequence of workload `name`'s shape, through
+    spla_append_kv_bulk and through the one-token kernel path (spla_append_kv), each chunk
+    timed alone with CUDA events after an L2 flush. Algorithmic bytes per chunk: the new
+    K and V read once and written once into the pool, the touched blocks' statistics, and
+    S, z, m read and written once."""
+    import torch
+    from block_sparse_linear_b200 import SplaDecodeCache
+    from workloads import feed_gpu, gen
+    w = gen.get(name)
+    cfg = feed_gpu.config_of(w)
+    hkv, d, bs, batch = w.num_kv_heads, w.head_dim, w.block_size, w.batch
+    mbp = (W + K) * n_tok // bs + 2
+    table = torch.arange(batch * mbp, dtype=torch.int32).reshape(batch, mbp)
+    g = torch.Generator(device=dev).manual_seed(5)
+    k = torch.randn((batch, n_tok, hkv, d), device=dev, generator=g).to(cfg.torch_dtype)
+    v = torch.randn((batch, n_tok, hkv, d), device=dev, generator=g).to(cfg.torch_dtype)
+    esz = k.element_size()
+    kv = 2 * batch * n_tok * hkv * d * esz
+    blocks = batch * hkv * (n_tok // bs + 1)
+    by = 2 * kv + blocks * 2 * d * 4 + 2 * batch * hkv * (d * d + 2 * d) * 4
+    out = {"workload": f"append of {n_tok} tokens per sequence, batch {batch}, {hkv} KV heads, "
+                       f"d {d}, block {bs}, {w.dtype}", "chunks": K, "bytes_per_chunk": by}
+    for bulk in (True, False):
+        cache = SplaDecodeCache(cfg, batch, table, batch * mbp, device=dev)
+        ts = []
+        for i in range(W + K):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            cache.append(k, v, bulk=bulk)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= W:
+                ts.append(e0.elapsed_time(e1))
+        ms = float(np.median(ts))
+        key = "bulk" if bulk else "one_token_path"
+        out[key] = {"ms_per_chunk": round(ms, 5),
+                    "tokens_per_s": round(batch * n_tok / (ms * 1e-3), 1),
+                    "dev_status": cache.status()}
+        if bulk:
+            out[key]["achieved_gbs"] = round(by / (ms * 1e-3) / 1e9, 1)
+        del cache
+    out["speedup"] = round(out["one_token_path"]["ms_per_chunk"] / out["bulk"]["ms_per_chunk"], 1)
+    torch.cuda.empty_cache()
+    return out
 
 
 def e2e_pass(w, cache, steps, s0, K, gamma, flush, dev, stream, ones):

@@ -83,6 +83,13 @@ static spla_status check_cache(const spla_cache* c) {
     return SPLA_OK;
 }
 
+// The append kernels read the pools back with 16-byte loads; the bulk merge moves
+// S rows as 16-byte vectors.
+static bool cache_aligned(const spla_cache* c) {
+    auto misaligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) != 0; };
+    return !(misaligned(c->k_pool) || misaligned(c->v_pool) || misaligned(c->S));
+}
+
 static CacheView view_of(const spla_params* p, const spla_cache* c) {
     CacheView v;
     v.k_pool = c->k_pool;
@@ -261,6 +268,7 @@ spla_status spla_append_kv(const spla_params* params, const spla_cache* cache, c
     if ((st = check_cache(cache)) != SPLA_OK) return st;
     if (max_new < 0 || !n_new) return SPLA_ERR_INVALID_ARG;
     if (max_new > 0 && (!k_new || !v_new)) return SPLA_ERR_INVALID_ARG;
+    if (!cache_aligned(cache)) return SPLA_ERR_INVALID_ARG;
     const CacheView v = view_of(params, cache);
     cudaError_t e = launch_append(v, params->dtype, k_new, v_new, n_new, max_new, dev_status,
                                   (cudaStream_t)stream);
@@ -295,7 +303,7 @@ spla_status spla_append_kv_bulk(const spla_params* params, const spla_cache* cac
     if (st != SPLA_OK) return st;
     if ((st = check_cache(cache)) != SPLA_OK) return st;
     if ((st = check_bulk(params, cache->batch, max_new)) != SPLA_OK) return st;
-    if (!n_new) return SPLA_ERR_INVALID_ARG;
+    if (!n_new || !cache_aligned(cache)) return SPLA_ERR_INVALID_ARG;
     const CacheView v = view_of(params, cache);
     cudaStream_t s = (cudaStream_t)stream;
     if (max_new == 0) {

@@ -55,23 +55,45 @@ __device__ void append_block(const CacheView& c, const T* k_new, const T* v_new,
     const int t_end = (int)((int64_t)L0 + n < blk_lo + bs ? (int64_t)L0 + n : blk_lo + bs);
     T* kp = (T*)c.k_pool + ((int64_t)phys * c.hkv + h) * bs * d;
     T* vp = (T*)c.v_pool + ((int64_t)phys * c.hkv + h) * bs * d;
-    // write the new tokens of this block
-    const int nw = (t_end - t_beg) * d;
-    for (int e = threadIdx.x; e < nw; e += blockDim.x) {
-        const int t = t_beg + e / d, i = e % d;
-        const int64_t src = (((int64_t)b * max_new + (t - L0)) * c.hkv + h) * d + i;
-        kp[(int64_t)(t - blk_lo) * d + i] = k_new[src];
-        vp[(int64_t)(t - blk_lo) * d + i] = v_new[src];
+    // write the new tokens of this block: 16-byte vectors when every buffer allows them
+    const bool vec = ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new) |
+                       reinterpret_cast<uintptr_t>(c.k_pool) |
+                       reinterpret_cast<uintptr_t>(c.v_pool)) & 15) == 0;
+    if (vec) {
+        constexpr int EPV = 16 / sizeof(T);
+        const int vpr = d / EPV;                     // vectors per token row
+        const int nv = (t_end - t_beg) * vpr;
+        for (int e = threadIdx.x; e < nv; e += blockDim.x) {
+            const int t = t_beg + e / vpr, u = e % vpr;
+            const int64_t src = (((int64_t)b * max_new + (t - L0)) * c.hkv + h) * d + u * EPV;
+            const int64_t dst = (int64_t)(t - blk_lo) * d + u * EPV;
+            const int4 kx = *reinterpret_cast<const int4*>(k_new + src);
+            const int4 vx = *reinterpret_cast<const int4*>(v_new + src);
+            *reinterpret_cast<int4*>(kp + dst) = kx;
+            *reinterpret_cast<int4*>(vp + dst) = vx;
+            const T* ke = reinterpret_cast<const T*>(&kx);
+#pragma unroll
+            for (int q = 0; q < EPV; ++q) ktile[dst + q] = to_f(ke[q]);   // staged for the statistics
+        }
+    } else {
+        const int nw = (t_end - t_beg) * d;
+        for (int e = threadIdx.x; e < nw; e += blockDim.x) {
+            const int t = t_beg + e / d, i = e % d;
+            const int64_t src = (((int64_t)b * max_new + (t - L0)) * c.hkv + h) * d + i;
+            kp[(int64_t)(t - blk_lo) * d + i] = k_new[src];
+            vp[(int64_t)(t - blk_lo) * d + i] = v_new[src];
+        }
     }
-    __syncthreads();
-    // statistics over all tokens now in the block: stage the keys in shared
-    // memory with coalesced loads, then two passes per dimension in fp64
+    // statistics over all tokens now in the block: the keys staged in shared memory
+    // (the new ones above when vectors were used, the older ones -- or all of them --
+    // read back from the pool with coalesced loads), then two passes per dimension in fp64
     const int nj = t_end - (int)blk_lo;
+    if (!vec) __syncthreads();                       // the scalar writes above, before reading back
     {
         // 16-byte loads, a batch of them in flight before any store (d is a multiple
         // of 64, so a block's nj*d keys split into whole vectors)
         constexpr int EPV = 16 / sizeof(T);
-        const int nvec = nj * d / EPV;
+        const int nvec = (vec ? t_beg - (int)blk_lo : nj) * d / EPV;
         const int4* src = reinterpret_cast<const int4*>(kp);
         constexpr int kBatch = 4;
         for (int v0 = threadIdx.x; v0 < nvec; v0 += kBatch * blockDim.x) {

@@ -21,7 +21,7 @@
 //                      split order (the result does not depend on timing).
 //
 // bulk_state_kernel roles: warp 0 issues the TMA loads (64-token tiles of K and V,
-// two 64-dimension boxes each, 128-byte swizzle, no multicast) into a two-stage
+// two 64-dimension boxes each, 128-byte swizzle, no multicast) into a three-stage
 // ring; warp 1 owns the tensor memory and issues the MMAs; warps 2..9 turn each
 // K tile into Phi in place. Phi is split into three bf16 parts (hi + mid + lo
 // carries 24 bits of its fp32 value, so the products lose nothing a fp32
@@ -35,7 +35,7 @@
 namespace spla {
 
 constexpr int kBulkTok = 64;                 // tokens per stage
-constexpr int kBulkStages = 2;
+constexpr int kBulkStages = 3;
 constexpr int kBulkTile = 16384;             // 64 tokens x 128 dims bf16 (two 8 KiB boxes)
 constexpr int kBulkStage = 4 * kBulkTile;    // Phi hi (in place of K), mid, lo, V
 constexpr int kBulkXformWarps = 8;
@@ -232,12 +232,21 @@ bulk_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
         float mx[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx[e] = -SPLA_INF;
-        for (int t = r0; t < ntok; t += 16) {
-            const uint4 q = *reinterpret_cast<const uint4*>(
-                k_new + (((int64_t)(row0 + t)) * hkv + h) * kBulkD + 8 * g);
-            const __nv_bfloat16* e8 = reinterpret_cast<const __nv_bfloat16*>(&q);
+        // eight loads in flight per thread before any of them is used
+        for (int t = r0; t < ntok; t += 16 * 8) {
+            uint4 q[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], __bfloat162float(e8[e]));
+            for (int u = 0; u < 8; ++u)
+                if (t + 16 * u < ntok)
+                    q[u] = *reinterpret_cast<const uint4*>(
+                        k_new + (((int64_t)(row0 + t + 16 * u)) * hkv + h) * kBulkD + 8 * g);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (t + 16 * u < ntok) {
+                    const __nv_bfloat16* e8 = reinterpret_cast<const __nv_bfloat16*>(&q[u]);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], __bfloat162float(e8[e]));
+                }
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) red[r0][8 * g + e] = mx[e];
@@ -363,7 +372,7 @@ bulk_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
 }
 
 // Rows [8 rg, 8 rg + 8) of S (and of z, m) of one (sequence, KV head): warp r owns
-// row 8 rg + r, lane l columns l + 32u.
+// row 8 rg + r, lane l columns 4l .. 4l + 3. Partials are added in split order.
 __global__ void __launch_bounds__(256)
 bulk_merge_kernel(CacheView c, const int32_t* n_new, int32_t max_new, int splits, int tsplit,
                   const float* __restrict__ part) {
@@ -376,29 +385,44 @@ bulk_merge_kernel(CacheView c, const int32_t* n_new, int32_t max_new, int splits
     const int32_t L0 = c.lens[b], n = n_new[b];
     if (n <= 0 || n > max_new) return;             // flagged by the block kernel
     if (L0 < 0 || (int64_t)L0 + n > (int64_t)c.mbp * c.bs) return;
-    const int d = kBulkD;
+    constexpr int d = kBulkD;
+    constexpr int64_t R = bulk_record_floats(d);
     const int nsp = min(splits, (n + tsplit - 1) / tsplit);
-    const float* rec0 = part + (int64_t)bh * splits * bulk_record_floats(d);
+    const float* rec0 = part + (int64_t)bh * splits * R;
     const int64_t gidx = (int64_t)bh * d + row;
     const float m_old = c.m[gidx];
     float m_new = m_old;
-    for (int sp = 0; sp < nsp; ++sp)
-        m_new = fmaxf(m_new, rec0[sp * bulk_record_floats(d) + d * d + d + row]);
+    for (int sp = lane; sp < nsp; sp += 32) m_new = fmaxf(m_new, rec0[sp * R + d * d + d + row]);
+    m_new = warp_max(m_new);
     const float f_old = (m_old == -SPLA_INF) ? 0.f : expf(m_old - m_new);
-    float* Srow = c.S + gidx * d;
-    float acc[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] = Srow[lane + 32 * u] * f_old;
+    float4* S4 = reinterpret_cast<float4*>(c.S + gidx * d) + lane;
+    float4 acc = *S4;
+    acc.x *= f_old; acc.y *= f_old; acc.z *= f_old; acc.w *= f_old;
     float zt = c.z[gidx] * f_old;
-    for (int sp = 0; sp < nsp; ++sp) {
-        const float* rec = rec0 + sp * bulk_record_floats(d);
-        const float f = expf(rec[d * d + d + row] - m_new);
+    constexpr int kBatch = 8;                       // partial rows in flight
+    for (int sp0 = 0; sp0 < nsp; sp0 += kBatch) {
+        float4 x[kBatch];
+        float mc[kBatch], zc[kBatch];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] = fmaf(rec[(int64_t)row * d + lane + 32 * u], f, acc[u]);
-        zt = fmaf(rec[d * d + row], f, zt);
+        for (int u = 0; u < kBatch; ++u)
+            if (sp0 + u < nsp) {
+                const float* rec = rec0 + (sp0 + u) * R;
+                x[u] = reinterpret_cast<const float4*>(rec + (int64_t)row * d)[lane];
+                mc[u] = rec[d * d + d + row];
+                zc[u] = rec[d * d + row];
+            }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+            if (sp0 + u < nsp) {
+                const float f = expf(mc[u] - m_new);
+                acc.x = fmaf(x[u].x, f, acc.x);
+                acc.y = fmaf(x[u].y, f, acc.y);
+                acc.z = fmaf(x[u].z, f, acc.z);
+                acc.w = fmaf(x[u].w, f, acc.w);
+                zt = fmaf(zc[u], f, zt);
+            }
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) Srow[lane + 32 * u] = acc[u];
+    *S4 = acc;
     if (lane == 0) {
         c.z[gidx] = zt;
         c.m[gidx] = m_new;

@@ -22,7 +22,8 @@
  *             cudaStream_t passed as void*; NULL = legacy default stream).
  *             spla_decode needs q and the cache's pools, statistics, S, z and
  *             m 16-byte aligned (it moves them with bulk copies and 16-byte
- *             loads) and returns SPLA_ERR_INVALID_ARG otherwise.
+ *             loads); the append calls need the pools and S 16-byte aligned.
+ *             Each returns SPLA_ERR_INVALID_ARG otherwise.
  *   Errors.   Argument errors are returned synchronously, before any CUDA
  *             call, and nothing is enqueued. Faults the kernels detect
  *             (a block-table entry out of range, a length past the table's

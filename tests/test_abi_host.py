@@ -151,3 +151,49 @@ def test_decode_rejects_misaligned_buffers(lib):
         c = _cache(**{field: FAKE + 4})
         assert lib.spla_decode(B(p), B(c), FAKE, None, FAKE, None, None, None, FAKE, need, None,
                                None) == _lib.SPLA_ERR_INVALID_ARG, field
+
+
+def test_append_rejects_misaligned_cache_buffers(lib):
+    """The append kernels read the pools back with 16-byte loads and the bulk merge moves S
+    rows as 16-byte vectors: misaligned pools or S are refused on the host."""
+    B = ctypes.byref
+    p = _params()
+    for field in ("k_pool", "v_pool", "S"):
+        c = _cache(**{field: FAKE + 8})
+        assert lib.spla_append_kv(B(p), B(c), FAKE, FAKE, FAKE, 4, None, None) == \
+            _lib.SPLA_ERR_INVALID_ARG, field
+        assert lib.spla_append_kv_bulk(B(p), B(c), FAKE, FAKE, FAKE, 4, FAKE, 1 << 40, None,
+                                       None) == _lib.SPLA_ERR_INVALID_ARG, field
+
+
+def test_bulk_append_host_checks(lib):
+    """spla_append_kv_bulk: bf16 and head_dim 128 only, aligned inputs, a large enough
+    workspace; its size query is a pure function of its arguments."""
+    B = ctypes.byref
+    p = _params()
+    c = _cache()
+    need = _lib.spla_append_bulk_workspace_size(p, 4, 8192)
+    assert need == _lib.spla_append_bulk_workspace_size(p, 4, 8192) > 0
+    assert _lib.spla_append_bulk_workspace_size(p, 4, 64) <= need
+    assert _lib.spla_append_bulk_workspace_size(p, 4, 0) == 0
+    for bad, code in ((_params(dtype=_lib.SPLA_F32), _lib.SPLA_ERR_UNSUPPORTED),
+                      (_params(head_dim=64, num_q_heads=8, num_kv_heads=2),
+                       _lib.SPLA_ERR_UNSUPPORTED)):
+        assert lib.spla_append_kv_bulk(B(bad), B(c), FAKE, FAKE, FAKE, 8192, FAKE, need, None,
+                                       None) == code
+        with pytest.raises(_lib.SplaError) as e:
+            _lib.spla_append_bulk_workspace_size(bad, 4, 8192)
+        assert e.value.status == code
+    # inputs: missing or misaligned
+    assert lib.spla_append_kv_bulk(B(p), B(c), None, FAKE, FAKE, 8192, FAKE, need, None,
+                                   None) == _lib.SPLA_ERR_INVALID_ARG
+    assert lib.spla_append_kv_bulk(B(p), B(c), FAKE, FAKE + 2, FAKE, 8192, FAKE, need, None,
+                                   None) == _lib.SPLA_ERR_INVALID_ARG
+    assert lib.spla_append_kv_bulk(B(p), B(c), FAKE, FAKE, None, 8192, FAKE, need, None,
+                                   None) == _lib.SPLA_ERR_INVALID_ARG
+    assert lib.spla_append_kv_bulk(B(p), B(c), FAKE, FAKE, FAKE, -1, FAKE, need, None,
+                                   None) == _lib.SPLA_ERR_INVALID_ARG
+    # workspace: missing, too small, misaligned
+    for ws, nbytes in ((None, need), (FAKE, need - 1), (FAKE + 8, need)):
+        assert lib.spla_append_kv_bulk(B(p), B(c), FAKE, FAKE, FAKE, 8192, ws, nbytes, None,
+                                       None) == _lib.SPLA_ERR_WORKSPACE
