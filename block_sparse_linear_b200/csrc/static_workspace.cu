@@ -13,6 +13,8 @@
 // kernel of the same call reads it, so no clearing is needed or done. Two calls
 // whose kernels overlap on the GPU (on different streams without ordering
 // between them) use the same words and race.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -31,19 +33,53 @@ __device__ __align__(256) unsigned char g_static_ws[SPLA_STATIC_WORKSPACE_BYTES]
 
 std::mutex g_setup_mutex;
 void* g_static_ws_ptr[kMaxDevices] = {};
+unsigned long long g_static_ws_ctx[kMaxDevices] = {};   // context the pointer belongs to
 
-// Device address of g_static_ws on device `dev`, which must be current. The
-// first call for a device looks it up; later calls return the stored pointer.
+// Unique id (for the life of the process) of the calling thread's current context,
+// through the driver entry points the runtime exposes; false when there is none.
+bool current_context_id(unsigned long long* id) {
+    using GetCurrentFn = CUresult (*)(CUcontext*);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_static_ws on device `dev`, which must be current. It is looked
+// up on the first call and again whenever the device's context has changed since
+// (a cudaDeviceReset reloads the module, and the array may move), or on every call
+// when the context cannot be identified.
 spla_status static_ws_for(int dev, void** out) {
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_static_ws_ptr[dev]) {
+    unsigned long long id = 0;
+    const bool known = current_context_id(&id);
+    if (!g_static_ws_ptr[dev] || !known || id != g_static_ws_ctx[dev]) {
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_static_ws);
         if (e != cudaSuccess) {
             spla::set_last_cuda_error((int32_t)e);
             return SPLA_ERR_CUDA;
         }
-        g_static_ws_ptr[dev] = p;
+        // the lookup made the device's context current if it was not yet
+        const bool now_known = current_context_id(&id);
+        g_static_ws_ptr[dev] = now_known ? p : nullptr;
+        g_static_ws_ctx[dev] = now_known ? id : 0;
+        *out = p;
+        return SPLA_OK;
     }
     *out = g_static_ws_ptr[dev];
     return SPLA_OK;

@@ -246,9 +246,11 @@ SPLA_API spla_status spla_decode(const spla_params* params, const spla_cache* ca
  *   SPLA_STATIC_WORKSPACE_BYTES returns SPLA_ERR_CAPACITY on the host, before
  *   any CUDA call, and enqueues nothing.
  *   First call per device: it looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current, and keeps it; make that
- *   first call before any stream capture on the device. A failed lookup
- *   returns SPLA_ERR_CUDA.
+ *   (cudaGetSymbolAddress) with that device current, and keeps it together
+ *   with the id of the device's context; a call that finds another context
+ *   current (after cudaDeviceReset, say, which reloads the module) looks it
+ *   up again. Make the first call in each context before any stream capture
+ *   on the device. A failed lookup returns SPLA_ERR_CUDA.
  *   Sharing: every call on a device uses the same array. Nothing in it needs
  *   to start at zero (each kernel writes its scratch before the next one reads
  *   it), so it is never cleared. Calls whose kernels overlap on the GPU (on

@@ -265,3 +265,34 @@ def test_full_size_sampled_heads_match_oracle(name):
         st = compare_all(res, oc, q, gamma, w)
         s = parity.check_ill(name, st, cache.status())
         print(name, step, s)
+
+
+def test_rla_cancellation_sets_unresolved_bit():
+    """The residual's denominator D - D~ sums the weights of the unselected tokens. Here the
+    one unselected block has keys at -200, whose exp(k - m) is 0 in fp32, so on the GPU
+    D - D~ is the difference of two fp32 evaluations of the same sum: its sign is rounding
+    noise. Wherever it is not positive the combine step returns o_rla = 0 and must raise
+    SPLA_DEV_RLA_UNRESOLVED; a head whose o_rla is exactly zero while a block went
+    unselected is such a head, and the bit is set exactly when one exists."""
+    from block_sparse_linear_b200 import SplaConfig, SplaDecodeCache, _lib
+    rng = np.random.default_rng(21)
+    batch, hq, hkv, d, bs, nb = 4, 16, 4, 128, 64, 8
+    cfg = SplaConfig(num_q_heads=hq, num_kv_heads=hkv, head_dim=d, block_size=bs, top_k=nb - 1)
+    table = torch.arange(batch * nb, dtype=torch.int32).reshape(batch, nb)
+    cache = SplaDecodeCache(cfg, batch, table, batch * nb, device="cuda")
+    k = rng.standard_normal((batch, nb * bs, hkv, d))
+    k[:, 3 * bs:4 * bs] = -200.0                    # block 3: weight exp(-200 - m) = 0 in fp32
+    v = rng.standard_normal((batch, nb * bs, hkv, d))
+    to = lambda a: torch.from_numpy(a).to(torch.bfloat16).cuda()
+    cache.append(to(k), to(v), bulk=False)
+    q = to(rng.standard_normal((batch, hq, d)))
+    out, sel, osp, orl = cache.new_outputs(debug=True)
+    cache.decode(q, None, out, sel, osp, orl)
+    torch.cuda.synchronize()
+    sel, orl = sel.cpu().numpy(), orl.cpu().numpy()
+    assert np.all((sel[..., :nb - 1] >= 0)) and not np.any(sel == 3)   # block 3 never selected
+    zero_heads = int(np.sum(np.all(orl == 0, axis=-1)))
+    status = cache.status()
+    assert status & ~_lib.SPLA_DEV_RLA_UNRESOLVED == 0, status
+    assert bool(status & _lib.SPLA_DEV_RLA_UNRESOLVED) == (zero_heads > 0), (status, zero_heads)
+    print(f"heads with D - D~ <= 0: {zero_heads} of {batch * hq}")
