@@ -269,7 +269,8 @@ def test_full_size_sampled_heads_match_oracle(name):
 
 def test_rla_cancellation_sets_unresolved_bit():
     """The residual's denominator D - D~ sums the weights of the unselected tokens. Here the
-    one unselected block has keys at -200, whose exp(k - m) is 0 in fp32, so on the GPU
+    one unselected block has keys at -200 (and every query is positive, so that block scores
+    lowest); its exp(k - m) is 0 in fp32, so on the GPU
     D - D~ is the difference of two fp32 evaluations of the same sum: its sign is rounding
     noise. Wherever it is not positive the combine step returns o_rla = 0 and must raise
     SPLA_DEV_RLA_UNRESOLVED; a head whose o_rla is exactly zero while a block went
@@ -285,7 +286,8 @@ def test_rla_cancellation_sets_unresolved_bit():
     v = rng.standard_normal((batch, nb * bs, hkv, d))
     to = lambda a: torch.from_numpy(a).to(torch.bfloat16).cuda()
     cache.append(to(k), to(v), bulk=False)
-    q = to(rng.standard_normal((batch, hq, d)))
+    # q > 0 in every dimension: block 3's mean of -200 gives it the lowest score of all
+    q = to(np.abs(rng.standard_normal((batch, hq, d))) + 0.1)
     out, sel, osp, orl = cache.new_outputs(debug=True)
     cache.decode(q, None, out, sel, osp, orl)
     torch.cuda.synchronize()
