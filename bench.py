@@ -429,7 +429,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def measure_prefill(name, dev, stream, flush, n_tok=8192, K=8, W=2):
+def measure_prefill(name, dev, stream, flush, n_tok=65536, K=4, W=2):
     """Bulk append of one n_tok-token chunk per sequence of workload `name`'s shape, through
     spla_append_kv_bulk and through the one-token kernel path (spla_append_kv), each chunk
     timed alone with CUDA events after an L2 flush. Algorithmic bytes per chunk: the new

@@ -63,17 +63,33 @@ __device__ void append_block(const CacheView& c, const T* k_new, const T* v_new,
         constexpr int EPV = 16 / sizeof(T);
         const int vpr = d / EPV;                     // vectors per token row
         const int nv = (t_end - t_beg) * vpr;
-        for (int e = threadIdx.x; e < nv; e += blockDim.x) {
-            const int t = t_beg + e / vpr, u = e % vpr;
-            const int64_t src = (((int64_t)b * max_new + (t - L0)) * c.hkv + h) * d + u * EPV;
-            const int64_t dst = (int64_t)(t - blk_lo) * d + u * EPV;
-            const int4 kx = *reinterpret_cast<const int4*>(k_new + src);
-            const int4 vx = *reinterpret_cast<const int4*>(v_new + src);
-            *reinterpret_cast<int4*>(kp + dst) = kx;
-            *reinterpret_cast<int4*>(vp + dst) = vx;
-            const T* ke = reinterpret_cast<const T*>(&kx);
+        // four K and four V vectors per thread in flight before any store
+        constexpr int kCopyBatch = 4;
+        for (int e0 = threadIdx.x; e0 < nv; e0 += kCopyBatch * blockDim.x) {
+            int4 kx[kCopyBatch], vx[kCopyBatch];
 #pragma unroll
-            for (int q = 0; q < EPV; ++q) ktile[dst + q] = to_f(ke[q]);   // staged for the statistics
+            for (int r = 0; r < kCopyBatch; ++r) {
+                const int e = e0 + r * blockDim.x;
+                if (e < nv) {
+                    const int t = t_beg + e / vpr, u = e % vpr;
+                    const int64_t src = (((int64_t)b * max_new + (t - L0)) * c.hkv + h) * d + u * EPV;
+                    kx[r] = *reinterpret_cast<const int4*>(k_new + src);
+                    vx[r] = *reinterpret_cast<const int4*>(v_new + src);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < kCopyBatch; ++r) {
+                const int e = e0 + r * blockDim.x;
+                if (e < nv) {
+                    const int t = t_beg + e / vpr, u = e % vpr;
+                    const int64_t dst = (int64_t)(t - blk_lo) * d + u * EPV;
+                    *reinterpret_cast<int4*>(kp + dst) = kx[r];
+                    *reinterpret_cast<int4*>(vp + dst) = vx[r];
+                    const T* ke = reinterpret_cast<const T*>(&kx[r]);
+#pragma unroll
+                    for (int q = 0; q < EPV; ++q) ktile[dst + q] = to_f(ke[q]);   // for the statistics
+                }
+            }
         }
     } else {
         const int nw = (t_end - t_beg) * d;
@@ -215,18 +231,22 @@ __device__ void append_rows(const CacheView& c, const T* k_new, const T* v_new,
 
 // One launch for both roles: CTAs x < nsb take blocks, the rest take row groups.
 template <typename T>
-__global__ void __launch_bounds__(256) append_kernel(CacheView c, const T* k_new, const T* v_new,
+__global__ void __launch_bounds__(256, 4) append_kernel(CacheView c, const T* k_new, const T* v_new,
                                                      const int32_t* n_new, int32_t max_new,
-                                                     int nsb, int32_t* status) {
+                                                     int nsb, int wait_last, int32_t* status) {
     extern __shared__ float ktile[];                 // [B][d], block role only
     const int b = blockIdx.y / c.hkv;
     const int h = blockIdx.y % c.hkv;
     pdl_trigger();
-    pdl_wait();
+    // wait_last: the kernel before this one already waited for everything this one
+    // reads and let it launch only then; waiting at the end keeps the kernels after
+    // this one ordered behind that predecessor too
+    if (!wait_last) pdl_wait();
     if ((int)blockIdx.x < nsb)
         append_block<T>(c, k_new, v_new, n_new, max_new, status, b, h, blockIdx.x, ktile);
     else
         append_rows<T>(c, k_new, v_new, n_new, max_new, b, h, blockIdx.x - nsb);
+    if (wait_last) pdl_wait();
 }
 
 __global__ void append_advance_kernel(CacheView c, const int32_t* n_new, int32_t max_new) {
@@ -261,7 +281,8 @@ cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s) {
 // The block role alone: tokens into the pool and the touched blocks' statistics.
 cudaError_t launch_append_blocks(const CacheView& c, int dtype, const void* k_new,
                                  const void* v_new, const int32_t* n_new, int32_t max_new,
-                                 int32_t* status, cudaStream_t s, bool with_rows) {
+                                 int32_t* status, cudaStream_t s, bool with_rows,
+                                 bool wait_last) {
     const int nsb = (max_new + c.bs - 1) / c.bs + 1;         // blocks a sequence's tokens can touch
     dim3 grid(nsb + (with_rows ? (c.d + 7) / 8 : 0), c.batch * c.hkv);
     const size_t smem = (size_t)c.bs * c.d * sizeof(float);
@@ -274,10 +295,10 @@ cudaError_t launch_append_blocks(const CacheView& c, int dtype, const void* k_ne
     if (dtype == SPLA_BF16) {
         using B16 = __nv_bfloat16;
         return launch_pdl(append_kernel<B16>, grid, dim3(256), smem, s, c, (const B16*)k_new,
-                          (const B16*)v_new, n_new, max_new, nsb, status);
+                          (const B16*)v_new, n_new, max_new, nsb, wait_last ? 1 : 0, status);
     }
     return launch_pdl(append_kernel<float>, grid, dim3(256), smem, s, c, (const float*)k_new,
-                      (const float*)v_new, n_new, max_new, nsb, status);
+                      (const float*)v_new, n_new, max_new, nsb, wait_last ? 1 : 0, status);
 }
 
 cudaError_t launch_append_advance(const CacheView& c, const int32_t* n_new, int32_t max_new,
@@ -290,7 +311,7 @@ cudaError_t launch_append(const CacheView& c, int dtype, const void* k_new, cons
                           cudaStream_t s) {
     if (max_new > 0) {
         cudaError_t e = launch_append_blocks(c, dtype, k_new, v_new, n_new, max_new, status, s,
-                                             /*with_rows=*/true);
+                                             /*with_rows=*/true, /*wait_last=*/false);
         if (e != cudaSuccess) return e;
     }
     return launch_append_advance(c, n_new, max_new, s);

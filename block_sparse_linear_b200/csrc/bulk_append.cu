@@ -9,8 +9,8 @@
 // The sum over t is Phi^T V with Phi[t][i] = e^{k_t,i - m_c,i}: an M = d by N = d
 // product over K = tokens, run on tcgen05 with the accumulator in tensor memory.
 //
-// Launches (after the block kernel has written the tokens into the pool and
-// recomputed the touched blocks' statistics):
+// Launches (the block kernel, which writes the tokens into the pool and recomputes
+// the touched blocks' statistics, runs beside the first):
 //   bulk_state_kernel  grid (splits, batch*Hkv), 320 threads: split c of a
 //                      (sequence, KV head) takes new tokens [c*T, (c+1)*T), finds
 //                      their per-dimension maximum m_c, and writes the partial
@@ -21,7 +21,7 @@
 //                      split order (the result does not depend on timing).
 //
 // bulk_state_kernel roles: warp 0 issues the TMA loads (64-token tiles of K and V,
-// two 64-dimension boxes each, 128-byte swizzle, no multicast) into a three-stage
+// two 64-dimension boxes each, 128-byte swizzle, no multicast) into a two-stage
 // ring; warp 1 owns the tensor memory and issues the MMAs; warps 2..9 turn each
 // K tile into Phi in place. Phi is split into three bf16 parts (hi + mid + lo
 // carries 24 bits of its fp32 value, so the products lose nothing a fp32
@@ -35,7 +35,7 @@
 namespace spla {
 
 constexpr int kBulkTok = 64;                 // tokens per stage
-constexpr int kBulkStages = 3;
+constexpr int kBulkStages = 2;
 constexpr int kBulkTile = 16384;             // 64 tokens x 128 dims bf16 (two 8 KiB boxes)
 constexpr int kBulkStage = 4 * kBulkTile;    // Phi hi (in place of K), mid, lo, V
 constexpr int kBulkXformWarps = 8;
@@ -145,11 +145,12 @@ bulk_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
     const int n = bulk_count(n_new, max_new, b);
     const int t0 = split * tsplit;
     const int ntok = max(0, min(n, t0 + tsplit) - t0);
+    // everything earlier on the stream (the previous call's merge reads this workspace,
+    // its length advance is what the block kernel after this one reads) is complete
+    // before this kernel lets the block kernel launch
+    pdl_wait();
     pdl_trigger();
-    if (ntok == 0) {                                // no partial: the merge skips this split
-        pdl_wait();
-        return;
-    }
+    if (ntok == 0) return;                          // no partial: the merge skips this split
     const int ntiles = (ntok + kBulkTok - 1) / kBulkTok;
     const int row0 = b * max_new + t0;              // first input row of this split
 
@@ -323,9 +324,6 @@ bulk_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&ready[s]);
         }
-        // partial record: written only after the previous kernel (which may still
-        // read this workspace) has completed
-        pdl_wait();
         float* rec = part + ((int64_t)bh * gridDim.x + split) * bulk_record_floats(kBulkD);
         asm volatile("bar.sync 1, %0;" :: "n"(kBulkXform));
 #pragma unroll
@@ -452,24 +450,28 @@ size_t bulk_workspace_bytes(int batch, int hkv, int d, int max_new) {
 
 cudaError_t launch_append_blocks(const CacheView& c, int dtype, const void* k_new,
                                  const void* v_new, const int32_t* n_new, int32_t max_new,
-                                 int32_t* status, cudaStream_t s, bool with_rows);
+                                 int32_t* status, cudaStream_t s, bool with_rows, bool wait_last);
 cudaError_t launch_append_advance(const CacheView& c, const int32_t* n_new, int32_t max_new,
                                   cudaStream_t s);
 
+// Order on the stream: state kernel (waits for everything before it, then lets the
+// next launch in), block kernel (runs beside it on the SMs' remaining shared memory
+// and registers; waits for the state kernel only at its end), merge, length advance.
 cudaError_t launch_append_bulk(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
                                const void* k_new, const void* v_new, const int32_t* n_new,
                                int32_t max_new, float* part, int32_t* status, cudaStream_t s) {
     int splits, tsplit;
     bulk_shape(c.batch, c.hkv, max_new, &splits, &tsplit);
-    cudaError_t e = launch_append_blocks(c, SPLA_BF16, k_new, v_new, n_new, max_new, status, s,
-                                         /*with_rows=*/false);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bulk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kBulkSmem);
+    cudaError_t e = cudaFuncSetAttribute(bulk_state_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kBulkSmem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(bulk_state_kernel, dim3(splits, c.batch * c.hkv), dim3(kBulkThreads), kBulkSmem,
                    s, tk, tv, (const __nv_bfloat16*)k_new, n_new, max_new, c.hkv, tsplit, part,
                    status);
+    if (e != cudaSuccess) return e;
+    e = launch_append_blocks(c, SPLA_BF16, k_new, v_new, n_new, max_new, status, s,
+                             /*with_rows=*/false, /*wait_last=*/true);
     if (e != cudaSuccess) return e;
     e = launch_pdl(bulk_merge_kernel, dim3(kBulkD / 8, c.batch * c.hkv), dim3(256), 0, s, c, n_new,
                    max_new, splits, tsplit, (const float*)part);
