@@ -552,7 +552,7 @@ __device__ __forceinline__ void rank_candidates(uint32_t* keys, const uint32_t* 
 //              bucket) buckets linear in key space, narrowed pass by pass.
 // Every step that reads what another warp wrote is one barrier apart; no loop
 // carries a dependency through shared memory.
-template <int NT>
+template <int NT, int MAXB>
 __global__ void __launch_bounds__(NT) select_kernel(CacheView c, int top_k, int n_sink,
                                                     int n_local, const float* scores, int ld,
                                                     uint32_t* bits, int nw, int32_t* nsel,
@@ -560,16 +560,16 @@ __global__ void __launch_bounds__(NT) select_kernel(CacheView c, int top_k, int 
                                                     KernelStamps* stamps) {
     constexpr int kSelThreads = NT;
     constexpr int kSelWarps = NT / 32;
-    constexpr int kWordsPerThread = SPLA_MAX_BLOCKS_PER_SEQ / 32 / NT;
+    constexpr int kWordsPerThread = MAXB / 32 / NT;
     constexpr int BPT = kBins / NT;             // histogram buckets per thread in the scans
-    static_assert(kWordsPerThread * 32 * NT == SPLA_MAX_BLOCKS_PER_SEQ, "bitset words per thread");
-    static_assert(SPLA_MAX_BLOCKS_PER_SEQ / NT <= 64, "candidate rounds fit a 64-bit mask");
+    static_assert(kWordsPerThread * 32 * NT == MAXB, "bitset words per thread");
+    static_assert(MAXB / NT <= 64, "candidate rounds fit a 64-bit mask");
     static_assert(BPT * NT == kBins, "buckets per thread");
     extern __shared__ __align__(16) unsigned char smem_sel[];
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem_sel);        // [mbp padded]
     __shared__ int hist[kBins];
-    __shared__ int wpre[SPLA_MAX_BLOCKS_PER_SEQ / 32];             // per-word counts, then prefixes
-    __shared__ uint32_t wword[SPLA_MAX_BLOCKS_PER_SEQ / 32];       // the bitset words
+    __shared__ int wpre[MAXB / 32];             // per-word counts, then prefixes
+    __shared__ uint32_t wword[MAXB / 32];       // the bitset words
     __shared__ uint32_t cand_key[kCandCap];
     __shared__ int cand_idx[kCandCap];
     __shared__ __align__(16) unsigned long long cand_c[kCandCap];   // key << 32 | ~index
@@ -933,17 +933,30 @@ cudaError_t launch_score(const CacheView& c, const CUtensorMap& tstats, int dtyp
                       : launch_score_t<64, float>(c, tstats, q, scale, first_order, scores, ld, gread, aw, stamps, status, s);
 }
 
+template <int NT, int MAXB>
+static cudaError_t launch_select_t(const CacheView& c, int top_k, int n_sink, int n_local,
+                                   const float* scores, int ld, uint32_t* bits, int nw,
+                                   int32_t* nsel, int32_t* sel_idx, int kcap,
+                                   KernelStamps* stamps, cudaStream_t s) {
+    const size_t smem = (size_t)((c.mbp + 31) / 32) * 32 * sizeof(uint32_t);
+    // static plus dynamic shared memory may pass the 48 KiB default
+    cudaError_t e = cudaFuncSetAttribute(select_kernel<NT, MAXB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(select_kernel<NT, MAXB>, dim3(c.batch * c.hq), dim3(NT), smem, s, c, top_k,
+                      n_sink, n_local, scores, ld, bits, nw, nsel, sel_idx, kcap, stamps);
+}
+
+// Threads per head by the table's capacity: a thread covers at most 64 blocks.
 cudaError_t launch_select(const CacheView& c, int top_k, int n_sink, int n_local,
                           const float* scores, int ld, uint32_t* bits, int nw, int32_t* nsel,
                           int32_t* sel_idx, int kcap, KernelStamps* stamps, cudaStream_t s) {
-    const size_t smem = (size_t)((c.mbp + 31) / 32) * 32 * sizeof(uint32_t);
-    const bool lng = c.mbp > kSelLongBlocks;
-    auto kern = lng ? select_kernel<kSelThreadsLong> : select_kernel<512>;
-    // static plus dynamic shared memory may pass the 48 KiB default
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(c.batch * c.hq), dim3(lng ? kSelThreadsLong : 512), smem, s, c,
-                      top_k, n_sink, n_local, scores, ld, bits, nw, nsel, sel_idx, kcap, stamps);
+    if (c.mbp <= kSelLongBlocks)
+        return launch_select_t<512, SPLA_MAX_BLOCKS_PER_SEQ>(c, top_k, n_sink, n_local, scores,
+                                                             ld, bits, nw, nsel, sel_idx, kcap,
+                                                             stamps, s);
+    return launch_select_t<kSelThreadsLong, SPLA_MAX_BLOCKS_PER_SEQ>(
+        c, top_k, n_sink, n_local, scores, ld, bits, nw, nsel, sel_idx, kcap, stamps, s);
 }
 
 }  // namespace spla
