@@ -88,7 +88,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.spla_decode_static_workspace.argtypes = [P, C, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.spla_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     lib.spla_profile_stamps.argtypes = [i32]
-    for f in ("spla_cache_init", "spla_append_kv", "spla_decode_workspace_size", "spla_decode",
+    for f in ("spla_cache_init", "spla_append_kv", "spla_append_kv_bulk",
+              "spla_append_bulk_workspace_size", "spla_decode_workspace_size", "spla_decode",
               "spla_decode_static_workspace", "spla_profile_events", "spla_profile_stamps"):
         getattr(lib, f).restype = ctypes.c_int
     lib.spla_status_string.argtypes = [ctypes.c_int]
