@@ -429,7 +429,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def measure_prefill(name, dev, stream, flush, n_tok=65536, K=4, W=2):
+def measure_prefill(name, dev, stream, flush, n_tok=65536, K=4, W=3):
     """Bulk append of one n_tok-token chunk per sequence of workload `name`'s shape, through
     spla_append_kv_bulk and through the one-token kernel path (spla_append_kv), each chunk
     timed alone with CUDA events after an L2 flush. Algorithmic bytes per chunk: the new
@@ -451,7 +451,8 @@ def measure_prefill(name, dev, stream, flush, n_tok=65536, K=4, W=2):
     blocks = batch * hkv * (n_tok // bs + 1)
     by = 2 * kv + blocks * 2 * d * 4 + 2 * batch * hkv * (d * d + 2 * d) * 4
     out = {"workload": f"append of {n_tok} tokens per sequence, batch {batch}, {hkv} KV heads, "
-                       f"d {d}, block {bs}, {w.dtype}", "chunks": K, "bytes_per_chunk": by}
+                       f"d {d}, block {bs}, {w.dtype}", "chunks": K, "warmup": W,
+           "l2": "flushed before every chunk", "bytes_per_chunk": by}
     for bulk in (True, False):
         cache = SplaDecodeCache(cfg, batch, table, batch * mbp, device=dev)
         ts = []
