@@ -35,6 +35,7 @@ SPLA_WS_STAMP_BYTES = 16384
 
 EXPORTS = ("spla_cache_init", "spla_append_kv", "spla_append_kv_bulk",
            "spla_append_bulk_workspace_size", "spla_decode_workspace_size", "spla_decode",
+           "spla_shard_candidates", "spla_shard_partials", "spla_shard_merge",
            "spla_decode_static_workspace", "spla_profile_events", "spla_profile_stamps",
            "spla_status_string", "spla_last_cuda_error", "spla_version")
 
@@ -86,11 +87,16 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.spla_decode_workspace_size.argtypes = [P, i32, i32, ctypes.POINTER(sz)]
     lib.spla_decode.argtypes = [P, C, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     lib.spla_decode_static_workspace.argtypes = [P, C, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.spla_shard_candidates.argtypes = [P, C, i32, vp, vp, vp, vp, sz, vp, vp]
+    lib.spla_shard_partials.argtypes = [P, C, i32, vp, vp, vp, i32, vp, vp, sz, vp, vp]
+    lib.spla_shard_merge.argtypes = [P, i32, vp, i32, vp, vp, vp, vp, vp, vp]
     lib.spla_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     lib.spla_profile_stamps.argtypes = [i32]
     for f in ("spla_cache_init", "spla_append_kv", "spla_append_kv_bulk",
               "spla_append_bulk_workspace_size", "spla_decode_workspace_size", "spla_decode",
-              "spla_decode_static_workspace", "spla_profile_events", "spla_profile_stamps"):
+           "spla_shard_candidates", "spla_shard_partials", "spla_shard_merge",
+              "spla_decode_static_workspace", "spla_profile_events", "spla_profile_stamps",
+              "spla_shard_candidates", "spla_shard_partials", "spla_shard_merge"):
         getattr(lib, f).restype = ctypes.c_int
     lib.spla_status_string.argtypes = [ctypes.c_int]
     lib.spla_status_string.restype = ctypes.c_char_p
@@ -131,6 +137,29 @@ def spla_append_bulk_workspace_size(params, batch, max_new) -> int:
            load().spla_append_bulk_workspace_size(ctypes.byref(params), batch, max_new,
                                                   ctypes.byref(n)))
     return n.value
+
+
+def spla_shard_candidates(params, cache, first_block, global_nb, q, cand, workspace,
+                          workspace_bytes, dev_status, stream=0):
+    _check("spla_shard_candidates",
+           load().spla_shard_candidates(ctypes.byref(params), ctypes.byref(cache), first_block,
+                                        global_nb, q, cand, workspace, workspace_bytes,
+                                        dev_status, stream))
+
+
+def spla_shard_partials(params, cache, first_block, global_nb, q, cand_all, nshards, part,
+                        workspace, workspace_bytes, dev_status, stream=0):
+    _check("spla_shard_partials",
+           load().spla_shard_partials(ctypes.byref(params), ctypes.byref(cache), first_block,
+                                      global_nb, q, cand_all, nshards, part, workspace,
+                                      workspace_bytes, dev_status, stream))
+
+
+def spla_shard_merge(params, batch, part_all, nshards, gamma, out, o_sparse, o_rla, dev_status,
+                     stream=0):
+    _check("spla_shard_merge",
+           load().spla_shard_merge(ctypes.byref(params), batch, part_all, nshards, gamma, out,
+                                   o_sparse, o_rla, dev_status, stream))
 
 
 def spla_decode_workspace_size(params, batch, max_blocks_per_seq) -> int:

@@ -15,6 +15,20 @@ cudaError_t launch_append_bulk(const CacheView& c, const CUtensorMap& tk, const 
                                const void* k_new, const void* v_new, const int32_t* n_new,
                                int32_t max_new, float* part, int32_t* status, cudaStream_t s);
 size_t bulk_workspace_bytes(int batch, int hkv, int d, int max_new);
+int shard_max_gathered();
+cudaError_t launch_shard_cand(const CacheView& c, const float* scores, int ld,
+                              const uint32_t* bits, int nw, int top_k, int n_sink, int n_local,
+                              int32_t first_block, const int32_t* global_nb, void* cand,
+                              int32_t* status, cudaStream_t s);
+cudaError_t launch_shard_mark(const CacheView& c, const float* scores, int ld,
+                              const void* cand_all, int nshards, int top_k, int n_sink,
+                              int n_local, int32_t first_block, const int32_t* global_nb,
+                              uint32_t* bits, int nw, int32_t* nsel, cudaStream_t s);
+cudaError_t launch_shard_partial(const CacheView& c, int dtype, const DecodeArgs& a,
+                                 const void* q, double* rec, cudaStream_t s);
+cudaError_t launch_shard_merge(int heads, int hq, int d, int dtype, const double* rec_all,
+                               int nshards, int no_rla, float eps, const float* gamma, void* out,
+                               float* o_sp, float* o_rl, int32_t* status, cudaStream_t s);
 cudaError_t launch_score(const CacheView& c, const CUtensorMap& tstats, int dtype, const void* q,
                          double scale, int first_order, float* scores, int ld, float* gread,
                          float* aw, KernelStamps* stamps, int32_t* status, cudaStream_t s);
@@ -420,6 +434,137 @@ spla_status spla_decode(const spla_params* params, const spla_cache* cache, cons
     prof_mark(4, s);
     prof_done(5, s);
     return SPLA_OK;
+}
+
+
+// ------------------------------------------------------------------ context-sharded decode
+// Checks shared by the two per-shard phases; fills the view, layout, scale.
+static spla_status shard_setup(const spla_params* params, const spla_cache* cache, const void* q,
+                               const int32_t* global_nb, int32_t first_block, void* workspace,
+                               size_t workspace_bytes, CacheView* v, DecodeLayout* L) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if ((st = check_cache(cache)) != SPLA_OK) return st;
+    if (!q || !global_nb || first_block < 0) return SPLA_ERR_INVALID_ARG;
+    auto misaligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) != 0; };
+    if (misaligned(q) || misaligned(cache->S) || misaligned(cache->z) || misaligned(cache->m) ||
+        misaligned(cache->blk_stats) || misaligned(cache->k_pool) || misaligned(cache->v_pool))
+        return SPLA_ERR_INVALID_ARG;
+    *L = layout_of(params, cache->batch, cache->max_blocks_per_seq);
+    if (!workspace || workspace_bytes < L->total) return SPLA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return SPLA_ERR_WORKSPACE;
+    *v = view_of(params, cache);
+    return SPLA_OK;
+}
+
+spla_status spla_shard_candidates(const spla_params* params, const spla_cache* cache,
+                                  int32_t first_block, const int32_t* global_nb, const void* q,
+                                  spla_candidate* cand, void* workspace, size_t workspace_bytes,
+                                  int32_t* dev_status, void* stream) {
+    CacheView v;
+    DecodeLayout L;
+    spla_status st = shard_setup(params, cache, q, global_nb, first_block, workspace,
+                                 workspace_bytes, &v, &L);
+    if (st != SPLA_OK) return st;
+    if (!cand) return SPLA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = static_cast<char*>(workspace);
+    float* scores = reinterpret_cast<float*>(ws + L.off_scores);
+    uint32_t* bits = reinterpret_cast<uint32_t*>(ws + L.off_bits);
+    int32_t* nsel = reinterpret_cast<int32_t*>(ws + L.off_nsel);
+    float* gread = reinterpret_cast<float*>(ws + L.off_gread);
+    float* aw_ws = reinterpret_cast<float*>(ws + L.off_aw);
+    const double scale = params->softmax_scale > 0.f ? (double)params->softmax_scale
+                                                     : 1.0 / sqrt((double)params->head_dim);
+    const int first_order = (params->flags & SPLA_FLAG_FIRST_ORDER) ? 1 : 0;
+    CUtensorMap tstats;
+    if (!make_stats_map(&tstats, v)) return cuda_fail(cudaErrorInvalidValue);
+    cudaError_t e = launch_score(v, tstats, params->dtype, q, scale, first_order, scores, L.ld,
+                                 gread, aw_ws, nullptr, dev_status, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    // the shard's best top_k + n_sink + n_local blocks, nothing forced: they hold its
+    // share of the sequence's top_k whatever the sink and local blocks are
+    e = launch_select(v, L.kcap, 0, 0, scores, L.ld, bits, L.nw, nsel, nullptr, L.kcap, nullptr, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_shard_cand(v, scores, L.ld, bits, L.nw, params->top_k, params->n_sink,
+                          params->n_local, first_block, global_nb, cand, dev_status, s);
+    return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
+}
+
+spla_status spla_shard_partials(const spla_params* params, const spla_cache* cache,
+                                int32_t first_block, const int32_t* global_nb, const void* q,
+                                const spla_candidate* cand_all, int32_t nshards, double* part,
+                                void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                void* stream) {
+    CacheView v;
+    DecodeLayout L;
+    spla_status st = shard_setup(params, cache, q, global_nb, first_block, workspace,
+                                 workspace_bytes, &v, &L);
+    if (st != SPLA_OK) return st;
+    if (!cand_all || !part || nshards < 1) return SPLA_ERR_INVALID_ARG;
+    if ((int64_t)nshards * params->top_k > shard_max_gathered()) return SPLA_ERR_CAPACITY;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = static_cast<char*>(workspace);
+    float* scores = reinterpret_cast<float*>(ws + L.off_scores);
+    uint32_t* bits = reinterpret_cast<uint32_t*>(ws + L.off_bits);
+    int32_t* nsel = reinterpret_cast<int32_t*>(ws + L.off_nsel);
+    const double scale = params->softmax_scale > 0.f ? (double)params->softmax_scale
+                                                     : 1.0 / sqrt((double)params->head_dim);
+    const bool use_mma = params->dtype == SPLA_BF16;
+    const size_t smem = use_mma ? mma_smem_for(v.d, v.bs, L.max_per)
+                                : simt_smem_for(v.d, v.bs, L.max_per);
+    if (smem > (size_t)kMaxSmem) return SPLA_ERR_CAPACITY;
+    cudaError_t e = launch_shard_mark(v, scores, L.ld, cand_all, nshards, params->top_k,
+                                      params->n_sink, params->n_local, first_block, global_nb,
+                                      bits, L.nw, nsel, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    DecodeArgs da;
+    da.q = q;
+    da.gamma = nullptr;
+    da.out = nullptr;
+    da.o_sp = nullptr;
+    da.o_rl = nullptr;
+    da.bits = bits;
+    da.nsel = nsel;
+    da.part = reinterpret_cast<float*>(ws + L.off_part);
+    da.gread = reinterpret_cast<float*>(ws + L.off_gread);
+    da.aw = reinterpret_cast<float*>(ws + L.off_aw);
+    da.stamps = nullptr;
+    da.status = dev_status;
+    da.nw = L.nw;
+    da.nsplit = L.nsplit;
+    da.max_per = L.max_per;
+    da.no_rla = (params->flags & SPLA_FLAG_NO_RLA) ? 1 : 0;
+    da.nrd = L.readout_parts;
+    da.sl2 = (float)(scale * 1.4426950408889634);
+    da.eps = params->rms_eps > 0.f ? params->rms_eps : 1e-6f;
+    if (use_mma) {
+        CUtensorMap tk, tv;
+        if (!make_pool_map(&tk, v.k_pool, v) || !make_pool_map(&tv, v.v_pool, v))
+            return cuda_fail(cudaErrorInvalidValue);
+        e = launch_decode_mma(v, tk, tv, da, s);
+    } else {
+        e = launch_decode_simt(v, params->dtype, da, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_shard_partial(v, params->dtype, da, q, part, s);
+    return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
+}
+
+spla_status spla_shard_merge(const spla_params* params, int32_t batch, const double* part_all,
+                             int32_t nshards, const float* rms_gamma, void* out,
+                             float* o_sparse_dbg, float* o_rla_dbg, int32_t* dev_status,
+                             void* stream) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if (batch <= 0 || nshards < 1 || !part_all || !out) return SPLA_ERR_INVALID_ARG;
+    const float eps = params->rms_eps > 0.f ? params->rms_eps : 1e-6f;
+    const int no_rla = (params->flags & SPLA_FLAG_NO_RLA) ? 1 : 0;
+    cudaError_t e = launch_shard_merge(batch * params->num_q_heads, params->num_q_heads,
+                                       params->head_dim, params->dtype, part_all, nshards, no_rla,
+                                       eps, rms_gamma, out, o_sparse_dbg, o_rla_dbg, dev_status,
+                                       (cudaStream_t)stream);
+    return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
 }
 
 }  // extern "C"

@@ -227,6 +227,60 @@ SPLA_API spla_status spla_decode(const spla_params* params, const spla_cache* ca
                         int32_t* dev_status, void* stream);
 
 /*
+ * Context-sharded decode (one long sequence over several GPUs, or several caches):
+ * the method's decode step split into three phases with an exchange between
+ * them. Shard s holds the global blocks [first_block, first_block +
+ * max_blocks_per_seq) of every sequence in a cache of its own (pools,
+ * statistics, and S, z, m over its own tokens; context_lens = its tokens);
+ * global_nb [batch] (device int32) is each sequence's total block count. The
+ * sink and local blocks are those of the whole sequence. Every shard passes the
+ * same params, batch and query q. The kept set equals the unsharded one: the
+ * sequence's top_k is the top_k of the union of the shards' local top_k. This
+ * is the library's own split of the step over devices (the pages describe the
+ * single-device step: section 2.1 selection, section 2.2 the residual by
+ * subtraction, section 2.3 the output).
+ *
+ * 1. spla_shard_candidates: scores this shard's blocks and writes, per
+ *    (sequence, query head), its best top_k blocks that are not sink or local
+ *    blocks, best first (score descending, ties to the lower global block),
+ *    padded with block = -1: cand [batch][Hq][top_k].
+ * 2. The caller gathers every shard's cand into cand_all [nshards][batch][Hq][top_k]
+ *    (an all-gather); nshards * top_k <= 4096.
+ * 3. spla_shard_partials: with the same workspace as step 1, untouched in
+ *    between, keeps this shard's forced blocks and those at or above the
+ *    sequence's top_k-th candidate, decodes them and writes one record per
+ *    (sequence, query head): part [batch][Hq][SPLA_SHARD_REC(d)] fp64.
+ * 4. The caller gathers every shard's part into part_all [nshards][batch][Hq][...].
+ * 5. spla_shard_merge: out (and the debug outputs) exactly as spla_decode
+ *    defines them, from part_all; any stream, no cache needed.
+ * The workspace is spla_decode_workspace_size(params, batch, max_blocks_per_seq)
+ * bytes. Argument checks and device faults as for spla_decode;
+ * SPLA_ERR_CAPACITY when nshards * top_k exceeds 4096.
+ */
+typedef struct {
+    float score;      /* the block's score (log of the Taylor estimate) */
+    int32_t block;    /* global block index, -1 for none */
+} spla_candidate;
+
+#define SPLA_SHARD_REC(d) (8 + 2 * (d))
+
+SPLA_API spla_status spla_shard_candidates(const spla_params* params, const spla_cache* cache,
+                                  int32_t first_block, const int32_t* global_nb,
+                                  const void* q, spla_candidate* cand, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+SPLA_API spla_status spla_shard_partials(const spla_params* params, const spla_cache* cache,
+                                int32_t first_block, const int32_t* global_nb, const void* q,
+                                const spla_candidate* cand_all, int32_t nshards, double* part,
+                                void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                void* stream);
+
+SPLA_API spla_status spla_shard_merge(const spla_params* params, int32_t batch,
+                             const double* part_all, int32_t nshards, const float* rms_gamma,
+                             void* out, float* o_sparse_dbg, float* o_rla_dbg,
+                             int32_t* dev_status, void* stream);
+
+/*
  * Bytes of the library-owned scratch that spla_decode_static_workspace uses
  * on each device (one file-scope __device__ array, 256-byte aligned).
  */

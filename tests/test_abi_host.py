@@ -197,3 +197,40 @@ def test_bulk_append_host_checks(lib):
     for ws, nbytes in ((None, need), (FAKE, need - 1), (FAKE + 8, need)):
         assert lib.spla_append_kv_bulk(B(p), B(c), FAKE, FAKE, FAKE, 8192, ws, nbytes, None,
                                        None) == _lib.SPLA_ERR_WORKSPACE
+
+
+def test_sharded_decode_host_checks(lib):
+    """spla_shard_*: missing buffers, a negative first block, a short workspace and too many
+    gathered candidates are refused on the host, before any CUDA call."""
+    B = ctypes.byref
+    p = _params()
+    c = _cache()
+    need = _lib.spla_decode_workspace_size(p, 4, 2064)
+    ok = dict(first=0, gnb=FAKE, q=FAKE, ws=FAKE, n=need)
+    args = lambda **kw: {**ok, **kw}
+
+    def cand(**kw):
+        a = args(**kw)
+        return lib.spla_shard_candidates(B(p), B(c), a["first"], a["gnb"], a["q"], FAKE, a["ws"],
+                                         a["n"], None, None)
+
+    def part(nshards=2, **kw):
+        a = args(**kw)
+        return lib.spla_shard_partials(B(p), B(c), a["first"], a["gnb"], a["q"], FAKE, nshards,
+                                       FAKE, a["ws"], a["n"], None, None)
+
+    for f in (cand, part):
+        assert f(first=-1) == _lib.SPLA_ERR_INVALID_ARG
+        assert f(gnb=None) == _lib.SPLA_ERR_INVALID_ARG
+        assert f(q=None) == _lib.SPLA_ERR_INVALID_ARG
+        assert f(q=FAKE + 4) == _lib.SPLA_ERR_INVALID_ARG
+        assert f(ws=None) == _lib.SPLA_ERR_WORKSPACE
+        assert f(n=need - 1) == _lib.SPLA_ERR_WORKSPACE
+    assert lib.spla_shard_candidates(B(p), B(c), 0, FAKE, FAKE, None, FAKE, need, None,
+                                     None) == _lib.SPLA_ERR_INVALID_ARG
+    assert part(nshards=0) == _lib.SPLA_ERR_INVALID_ARG
+    assert part(nshards=4096 // p.top_k + 1) == _lib.SPLA_ERR_CAPACITY
+    assert lib.spla_shard_merge(B(p), 4, None, 2, None, FAKE, None, None, None,
+                                None) == _lib.SPLA_ERR_INVALID_ARG
+    assert lib.spla_shard_merge(B(p), 0, FAKE, 2, None, FAKE, None, None, None,
+                                None) == _lib.SPLA_ERR_INVALID_ARG

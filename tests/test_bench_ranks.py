@@ -76,3 +76,34 @@ def test_oracle_sample_stays_inside_the_reserved_capacity():
     assert n == 8
     *_, n = bench.oracle_sample(w, 0.0, steps=20)
     assert n == 8
+
+
+def _gather_main(rank, world, port, out):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from block_sparse_linear_b200.sharded import dist_gather
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        # this rank's two shards' candidate rows, marked with the global shard index
+        local = torch.stack([torch.full((3, 2), 2 * rank + i, dtype=torch.int32) for i in range(2)])
+        out[rank] = dist_gather(local).tolist()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_decode_gather_orders_shards_by_rank_gloo_world_2():
+    """The all-gather between the sharded decode's phases stacks every rank's shards in
+    global shard order (rank-major), as spla_shard_partials and spla_shard_merge expect."""
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_gather_main, args=(2, port, out), nprocs=2, join=True)
+        got = dict(out)
+    want = [[[s, s]] * 3 for s in range(4)]
+    assert got[0] == got[1] == want
