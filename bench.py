@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shards", type=int, default=0,
+                    help="also time the context-sharded decode with the workload's sequences "
+                         "split into this many shard caches on this GPU")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the bulk-append (prefill chunk) measurement")
     ap.add_argument("--also", default="cfg4",
@@ -371,6 +374,7 @@ def run_ours(args):
         extra = (wx, mx, Kx)
 
     prefill = measure_prefill("cfg4", dev, stream, flush) if not args.no_prefill else None
+    sharded = measure_sharded(w, args.shards, K, W, dev, stream, flush) if args.shards > 0 else None
 
     # ---- max over ranks (the same single collective on every rank)
     t_max, e2e_ms, tx_max = max_over_ranks(
@@ -415,6 +419,8 @@ def run_ours(args):
                 "unit": UNIT, "roofline": sx["roofline"], "step_hbm": sx["step_roofline"],
                 "kernels_ms": sx["kernels_ms"], "dev_status": mx["status"],
                 "clocks": mx["clocks"]}
+        if sharded:
+            res["sharded_emulation"] = sharded
         if prefill:
             hbm_p = hbm
             prefill["bulk"]["frac_of_measured_peak" if peak_kind == "measured"
@@ -476,6 +482,103 @@ def measure_prefill(name, dev, stream, flush, n_tok=65536, K=4, W=3):
     out["speedup"] = round(out["one_token_path"]["ms_per_chunk"] / out["bulk"]["ms_per_chunk"], 1)
     torch.cuda.empty_cache()
     return out
+
+
+def measure_sharded(w, nshards, K, W, dev, stream, flush):
+    """The context-sharded decode with each sequence's blocks split over nshards caches on
+    this GPU (shard s holds global blocks [s*bps, (s+1)*bps)). Per step, after an L2 flush,
+    CUDA events around every shard's candidates call, every shard's partials call and the
+    merge: a rank of an nshards-GPU run would spend one shard's two phases, the merge and
+    two all-gathers (not timed here: one GPU)."""
+    import math
+
+    import torch
+    from block_sparse_linear_b200 import SplaDecodeCache, _lib
+    from block_sparse_linear_b200.sharded import rec_doubles
+    from workloads import feed_gpu, gen
+    cfg = feed_gpu.config_of(w)
+    bs, hkv, d, hq, k = w.block_size, w.num_kv_heads, w.head_dim, w.num_q_heads, w.top_k
+    nbg = [math.ceil(L / bs) for L in w.context_lens]
+    bps = math.ceil(max(nbg) / nshards)
+    span = bps * bs
+    shards = []
+    for s in range(nshards):
+        table = torch.arange(w.batch * bps, dtype=torch.int32).reshape(w.batch, bps)
+        shards.append((SplaDecodeCache(cfg, w.batch, table, w.batch * bps, device=dev), s * bps))
+    ct, dt = gen.CHUNK_TOKENS, cfg.torch_dtype
+    for c, chunk in gen.iter_prefix(w):
+        t0 = c * ct
+        for s, (cache, _) in enumerate(shards):
+            lo, hi = max(s * span, t0), min((s + 1) * span, t0 + ct)
+            if lo >= hi:
+                continue
+            parts = [(K[lo - t0:hi - t0], V[lo - t0:hi - t0]) for K, V in chunk]
+            counts = [int(p[0].shape[0]) for p in parts]
+            if max(counts) == 0:
+                continue
+            hk = torch.zeros((w.batch, max(counts), hkv, d), dtype=dt)
+            hv = torch.zeros_like(hk)
+            for b, (Kp, Vp) in enumerate(parts):
+                hk[b, :len(Kp)] = torch.from_numpy(Kp).to(dt)
+                hv[b, :len(Vp)] = torch.from_numpy(Vp).to(dt)
+            cache.append(hk.to(dev), hv.to(dev), torch.tensor(counts, dtype=torch.int32,
+                                                              device=dev))
+    torch.cuda.synchronize(dev)
+    q = torch.from_numpy(gen.query(w, 0)).to(dt).to(dev)
+    gamma = torch.ones((hq, d), dtype=torch.float32, device=dev)
+    gnb = torch.tensor(nbg, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    cand = torch.empty((nshards, w.batch, hq, k, 2), dtype=torch.int32, device=dev)
+    part = torch.empty((nshards, w.batch, hq, rec_doubles(d)), dtype=torch.float64, device=dev)
+    st = stream.cuda_stream
+
+    def step(evs=None):
+        rec = (lambda i: evs[i].record(stream)) if evs else (lambda i: None)
+        for i, (cache, first) in enumerate(shards):
+            rec(i)
+            _lib.spla_shard_candidates(cache.params, cache.c, first, gnb.data_ptr(), q.data_ptr(),
+                                       cand[i].data_ptr(), cache.workspace.data_ptr(),
+                                       cache.ws_bytes, cache.dev_status.data_ptr(), st)
+        for i, (cache, first) in enumerate(shards):
+            rec(nshards + i)
+            _lib.spla_shard_partials(cache.params, cache.c, first, gnb.data_ptr(), q.data_ptr(),
+                                     cand.data_ptr(), nshards, part[i].data_ptr(),
+                                     cache.workspace.data_ptr(), cache.ws_bytes,
+                                     cache.dev_status.data_ptr(), st)
+        rec(2 * nshards)
+        _lib.spla_shard_merge(shards[0][0].params, w.batch, part.data_ptr(), nshards,
+                              gamma.data_ptr(), out.data_ptr(), 0, 0,
+                              shards[0][0].dev_status.data_ptr(), st)
+        rec(2 * nshards + 1)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize(dev)
+    cand_ms, part_ms, merge_ms = [], [], []
+    for _ in range(K):
+        flush()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nshards + 2)]
+        step(evs)
+        torch.cuda.synchronize(dev)
+        t = [evs[i].elapsed_time(evs[i + 1]) for i in range(2 * nshards + 1)]
+        cand_ms += t[:nshards]
+        part_ms += t[nshards:2 * nshards]
+        merge_ms.append(t[2 * nshards])
+    status = 0
+    for cache, _ in shards:
+        status |= cache.status()
+    res = {"shards": nshards, "blocks_per_shard": bps, "steps": K, "warmup": W,
+           "l2": "flushed before every step",
+           "candidates_ms_per_shard": round(float(np.median(cand_ms)), 5),
+           "partials_ms_per_shard": round(float(np.median(part_ms)), 5),
+           "merge_ms": round(float(np.median(merge_ms)), 5),
+           "one_rank_ms": round(float(np.median(cand_ms) + np.median(part_ms) +
+                                      np.median(merge_ms)), 5),
+           "dev_status": status,
+           "not_timed": "the two all-gathers (NCCL) between the phases: one GPU"}
+    del shards
+    torch.cuda.empty_cache()
+    return res
 
 
 def e2e_pass(w, cache, steps, s0, K, gamma, flush, dev, stream, ones):
