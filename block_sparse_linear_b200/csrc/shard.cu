@@ -306,8 +306,11 @@ shard_partial_kernel(CacheView c, const DecodeArgs a, const T* q, double* rec_ou
 // One warp per (sequence, query head), lane l holding columns [l d/32, (l+1) d/32):
 // log-sum-exp merge of the shards' softmax parts, their residual parts rescaled
 // by exp(c_s - C) (C the largest c of a shard holding tokens) and added, the
-// subtraction, RMSNorm and the output.
-constexpr int kShardMergeWarps = 4;
+// subtraction, RMSNorm and the output. Lane s reads shard s's header (shards
+// past 32 in further rounds), so the maxima need one round trip; the records'
+// columns follow, four shards' loads in flight at a time.
+constexpr int kShardMergeWarps = 1;
+constexpr int kShardMergeBatch = 4;
 
 template <int D, typename T>
 __global__ void __launch_bounds__(kShardMergeWarps * 32)
@@ -321,28 +324,57 @@ shard_merge_kernel(int heads, int hq_count, const double* rec_all, int nshards, 
     pdl_wait();
     if (head >= heads) return;
     const int hq = head % hq_count;
+    auto rec = [&](int s) { return rec_all + ((int64_t)s * heads + head) * R; };
     double M = -INFINITY, C = -INFINITY, kept = 0.0, nblk = 0.0, ntok = 0.0;
-    for (int s = 0; s < nshards; ++s) {
-        const double* r = rec_all + ((int64_t)s * heads + head) * R;
-        M = fmax(M, r[0]);
-        if (r[6] > 0.0) C = fmax(C, r[2]);
-        kept += r[4];
-        nblk += r[5];
-        ntok += r[6];
+    for (int s = lane; s < nshards; s += 32) {
+        const double* r = rec(s);
+        const double m = r[0], cc = r[2], kk = r[4], nb = r[5], nt = r[6];
+        M = fmax(M, m);
+        if (nt > 0.0) C = fmax(C, cc);
+        kept += kk;
+        nblk += nb;
+        ntok += nt;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        M = fmax(M, __shfl_xor_sync(0xffffffffu, M, o));
+        C = fmax(C, __shfl_xor_sync(0xffffffffu, C, o));
+        kept += __shfl_xor_sync(0xffffffffu, kept, o);
+        nblk += __shfl_xor_sync(0xffffffffu, nblk, o);
+        ntok += __shfl_xor_sync(0xffffffffu, ntok, o);
     }
     double l = 0.0, rD = 0.0, o[CPL], rN[CPL];
 #pragma unroll
     for (int e = 0; e < CPL; ++e) { o[e] = 0.0; rN[e] = 0.0; }
-    for (int s = 0; s < nshards; ++s) {
-        const double* r = rec_all + ((int64_t)s * heads + head) * R;
-        const double f = (M == -INFINITY || r[0] == -INFINITY) ? 0.0 : exp2(r[0] - M);
-        const double w = (r[6] > 0.0 && C != -INFINITY) ? exp(r[2] - C) : 0.0;
-        l += r[1] * f;
-        rD += r[3] * w;
+    for (int s0 = 0; s0 < nshards; s0 += kShardMergeBatch) {
+        double hm[kShardMergeBatch], hl[kShardMergeBatch], hc[kShardMergeBatch],
+            hd[kShardMergeBatch], ht[kShardMergeBatch];
+        double xo[kShardMergeBatch][CPL], xn[kShardMergeBatch][CPL];
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) {
-            o[e] += r[8 + lane * CPL + e] * f;
-            rN[e] += r[8 + D + lane * CPL + e] * w;
+        for (int u = 0; u < kShardMergeBatch; ++u) {
+            if (s0 + u < nshards) {
+                const double* r = rec(s0 + u);
+                hm[u] = r[0]; hl[u] = r[1]; hc[u] = r[2]; hd[u] = r[3]; ht[u] = r[6];
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    xo[u][e] = r[8 + lane * CPL + e];
+                    xn[u][e] = r[8 + D + lane * CPL + e];
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kShardMergeBatch; ++u) {
+            if (s0 + u < nshards) {
+                const double f = (M == -INFINITY || hm[u] == -INFINITY) ? 0.0 : exp2(hm[u] - M);
+                const double w = (ht[u] > 0.0 && C != -INFINITY) ? exp(hc[u] - C) : 0.0;
+                l += hl[u] * f;
+                rD += hd[u] * w;
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    o[e] += xo[u][e] * f;
+                    rN[e] += xn[u][e] * w;
+                }
+            }
         }
     }
     const bool off = no_rla || kept >= nblk || ntok == 0.0;
