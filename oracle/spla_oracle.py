@@ -22,6 +22,9 @@ site repeats it):
 * section 2.3 "Architecture and Integration": parameter-free exponential
   feature map; output = gated sum of the sparse and RLA outputs with an RMS
   norm (whose scale is the only new parameter) on the RLA output. -> combine
+* the same sections in block-causal form (each query attends to the tokens up
+  to its own, its own block exactly, earlier blocks selected or covered by the
+  residual): -> block_causal_forward, linear_attention
 
 Readings where the pages leave a step open (the CUDA path makes the same ones):
  1. logits are q.k/sqrt(d); the Taylor score approximates the mass of those
@@ -243,6 +246,65 @@ def decode_head(q: np.ndarray, g: GroupState, p: OracleParams, gamma: np.ndarray
         o_rla = rla(N, D, Ns, Ds, all_sel)
     out = combine(o_sparse, o_rla, np.asarray(gamma, np.float64), p.rms_eps)
     return dict(out=out, o_sparse=o_sparse, o_rla=o_rla, sel=sel, scores=scores, n_blocks=nb)
+
+
+# ----------------------------------------------------------------------------- block-causal
+def linear_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """Normalised linear attention with phi = exp over the given tokens, evaluated directly:
+    sum_t w_t v_t / sum_t w_t, w_t = phi(q).phi(k_t) = sum_i exp(q_i + k_t,i), formed in
+    log space (each w_t by a log-sum-exp over i, then all w_t scaled by their maximum)."""
+    if K.shape[0] == 0:
+        return np.zeros(V.shape[1])
+    x = np.asarray(q, np.float64)[None, :] + K          # [n][d]: q_i + k_t,i
+    xm = x.max(axis=1, keepdims=True)
+    lw = xm[:, 0] + np.log(np.exp(x - xm).sum(axis=1))  # log w_t
+    w = np.exp(lw - lw.max())
+    return (w @ V) / w.sum()
+
+
+def block_causal_forward(K: np.ndarray, V: np.ndarray, Q: np.ndarray, p: OracleParams,
+                         gamma: np.ndarray) -> dict:
+    """The block-causal form of the method over one KV head's sequence: query t (row t of
+    Q [L][G][d], G heads of the group) sees tokens 0..t. Its own block J = t // B is
+    attended exactly (causally: tokens J*B..t); the complete earlier blocks 0..J-1 are
+    the candidates, scored by the Taylor estimate and the top_k of them (after any sink
+    blocks) attended exactly; the candidates left out are covered by linear attention
+    over their tokens (section 2.2: the residual is linear attention over the unselected
+    blocks), evaluated here directly from those tokens; out as in section 2.3.
+    Returns out, o_sparse, o_rla [L][G][d] and sel (list of kept candidate arrays)."""
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    L, d = K.shape
+    G = Q.shape[1]
+    B = p.block_size
+    n_all, mean_all, var_all = block_stats(K[:(L // B) * B], B) if L >= B else (
+        np.zeros(0), np.zeros((0, d)), np.zeros((0, d)))
+    res = {k: np.zeros((L, G, d)) for k in ("out", "o_sparse", "o_rla")}
+    sels = []
+    for t in range(L):
+        J = t // B
+        row = []
+        for g in range(G):
+            q = np.asarray(Q[t, g], np.float64)
+            sel = np.zeros(0, np.int64)
+            if J > 0:
+                scores = block_scores(q, n_all[:J], mean_all[:J], var_all[:J], p.scale,
+                                      p.first_order)
+                sel = select_blocks(scores, p.top_k, p.n_sink, 0)
+            tokens = np.concatenate([_tokens_of(sel, B, J * B),
+                                     np.arange(J * B, t + 1)]).astype(np.int64)
+            o_sparse = sparse_attention(q, K[:t + 1], V[:t + 1], tokens, p.scale)
+            left = np.setdiff1d(np.arange(J * B), _tokens_of(sel, B, J * B))
+            o_rla = np.zeros(d) if (p.no_rla or len(left) == 0) else \
+                linear_attention(q, K[left], V[left])
+            res["out"][t, g] = combine(o_sparse, o_rla, np.asarray(gamma[g], np.float64),
+                                       p.rms_eps)
+            res["o_sparse"][t, g] = o_sparse
+            res["o_rla"][t, g] = o_rla
+            row.append(sel)
+        sels.append(row)
+    res["sel"] = sels
+    return res
 
 
 class OracleCache:

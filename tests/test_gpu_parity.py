@@ -298,3 +298,46 @@ def test_rla_cancellation_sets_unresolved_bit():
     assert status & ~_lib.SPLA_DEV_RLA_UNRESOLVED == 0, status
     assert bool(status & _lib.SPLA_DEV_RLA_UNRESOLVED) == (zero_heads > 0), (status, zero_heads)
     print(f"heads with D - D~ <= 0: {zero_heads} of {batch * hq}")
+
+
+@pytest.mark.parametrize("n_sink", [0, 1])
+def test_block_causal_forward_by_decode_steps(n_sink):
+    """The block-causal form over a 330-token sequence: per token, a one-token append and a
+    decode with the current block kept as a local block (n_local = 1), against the
+    oracle's decode step at every position (which equals its block-causal form row by
+    row: tests/test_oracle_pins.py) and against that form directly."""
+    from block_sparse_linear_b200 import SplaConfig, SplaDecodeCache
+    rng = np.random.default_rng(31 + n_sink)
+    L, hq, d, bs = 330, 4, 128, 64
+    nb = -(-L // bs)
+    cfg = SplaConfig(num_q_heads=hq, num_kv_heads=1, head_dim=d, block_size=bs, top_k=2,
+                     n_sink=n_sink, n_local=1)
+    off = np.repeat(rng.normal(0.0, 0.5, (nb, d)), bs, axis=0)[:L]
+    to16 = lambda a: torch.from_numpy(a).to(torch.bfloat16)
+    K = to16(rng.standard_normal((L, d)) + off).double().numpy()
+    V = to16(rng.standard_normal((L, d)) + off).double().numpy()
+    Q = to16(rng.standard_normal((L, hq, d))).double().numpy()
+    gamma = rng.uniform(0.5, 1.5, (hq, d))
+    table = torch.arange(nb, dtype=torch.int32).reshape(1, nb)
+    cache = SplaDecodeCache(cfg, 1, table, nb, device="cuda")
+    p = so.OracleParams(num_q_heads=hq, num_kv_heads=1, head_dim=d, block_size=bs, top_k=2,
+                        n_sink=n_sink, n_local=1)
+    oc = so.OracleCache(p, 1)
+    form = so.block_causal_forward(K, V, Q, so.OracleParams(**{**p.__dict__, "n_local": 0}),
+                                   gamma)
+    g_t = torch.from_numpy(gamma).float().cuda()
+    out, sel, osp, orl = cache.new_outputs(debug=True)
+    stats = []
+    for t in range(L):
+        kt = to16(K[t][None, None, None]).cuda()
+        cache.append(kt, to16(V[t][None, None, None]).cuda())
+        cache.decode(to16(Q[t][None]).cuda(), g_t, out, sel, osp, orl)
+        oc.append_group(0, 0, K[t:t + 1], V[t:t + 1])
+        res = {"out": out.float().cpu().numpy()[0], "sel": sel.cpu().numpy()[0],
+               "o_sparse": osp.cpu().numpy()[0], "o_rla": orl.cpu().numpy()[0]}
+        for h in range(hq):
+            stats.append(parity.compare_head({k: v[h] for k, v in res.items()}, oc, Q[t][None],
+                                             gamma, 0, h, "bf16"))
+            np.testing.assert_allclose(res["o_sparse"][h], form["o_sparse"][t, h], atol=2e-2)
+    s = parity.check_ill("cfg2", stats, cache.status())
+    print("block-causal", n_sink, s)

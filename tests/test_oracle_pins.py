@@ -281,3 +281,54 @@ def test_planted_blocks_are_selected_in_the_small_fp32_workload():
     for (b, h), r in res.items():
         assert set(planted.tolist()) <= set(r["sel"].tolist()), (h, planted, r["sel"])
         assert len(r["sel"]) == w.top_k
+
+
+# ----------------------------------------------------------------------------- block-causal form
+def _bc_case(L=37, d=8, B=4, G=2, top_k=2, n_sink=0, seed=5):
+    rng = np.random.default_rng(seed)
+    K = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    Q = rng.standard_normal((L, G, d))
+    p = so.OracleParams(num_q_heads=G, num_kv_heads=1, head_dim=d, block_size=B, top_k=top_k,
+                        n_sink=n_sink)
+    return K, V, Q, p
+
+
+def test_block_causal_with_every_block_kept_is_causal_softmax_attention():
+    """top_k above every block count: no residual, and each query's exact part is causal
+    softmax attention over tokens 0..t (torch SDPA with a causal mask, fp64)."""
+    K, V, Q, p = _bc_case(top_k=100)
+    r = so.block_causal_forward(K, V, Q, p, np.ones((2, 8)))
+    assert np.all(r["o_rla"] == 0)
+    for g in range(2):
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q[:, g])[None, None], torch.from_numpy(K)[None, None],
+            torch.from_numpy(V)[None, None], is_causal=True, scale=p.scale)[0, 0].numpy()
+        np.testing.assert_allclose(r["o_sparse"][:, g], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_attention_equals_the_unscaled_formula():
+    rng = np.random.default_rng(2)
+    q, K, V = rng.standard_normal(6), rng.standard_normal((9, 6)), rng.standard_normal((9, 6))
+    w = np.exp(K) @ np.exp(q)                      # phi(q).phi(k_t), small values
+    np.testing.assert_allclose(so.linear_attention(q, K, V), (w @ V) / w.sum(), rtol=1e-12)
+
+
+@pytest.mark.parametrize("n_sink", [0, 1])
+def test_block_causal_row_is_the_decode_step_with_a_local_block(n_sink):
+    """Row t of the block-causal form equals a decode step over tokens 0..t with the last
+    (current) block kept as a local block: the state-subtraction residual equals the
+    direct one over the candidates left out, and the kept sets agree."""
+    K, V, Q, p = _bc_case(n_sink=n_sink)
+    gamma = np.linspace(0.5, 1.5, 16).reshape(2, 8)
+    r = so.block_causal_forward(K, V, Q, p, gamma)
+    pl = so.OracleParams(**{**p.__dict__, "n_local": 1})
+    g = so.GroupState(8)
+    for t in range(K.shape[0]):
+        so.append(g, K[t:t + 1], V[t:t + 1])
+        J = t // p.block_size
+        for h in range(2):
+            ref = so.decode_head(Q[t, h], g, pl, gamma[h])
+            assert list(ref["sel"]) == sorted(set(r["sel"][t][h].tolist()) | {J})
+            for key in ("out", "o_sparse", "o_rla"):
+                np.testing.assert_allclose(r[key][t, h], ref[key], rtol=1e-9, atol=1e-12)
