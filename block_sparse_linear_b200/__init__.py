@@ -91,11 +91,36 @@ class SplaDecodeCache:
                                      device=dev)
         self._n_new = torch.zeros((batch,), dtype=torch.int32, device=dev)
         self._bulk_ws = None
+        self._bc_ws = None
         spla_cache_init(self.params, self.c, self._stream(stream))
 
     def _stream(self, stream=None) -> int:
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         return s.cuda_stream
+
+    def block_causal_forward(self, k_all: torch.Tensor, v_all: torch.Tensor, q_all: torch.Tensor,
+                             gamma: torch.Tensor = None, out: torch.Tensor = None,
+                             o_sparse: torch.Tensor = None, o_rla: torch.Tensor = None,
+                             stream=None) -> torch.Tensor:
+        """The block-causal form over the sequences this cache holds (appended from k_all,
+        v_all [batch][max_len][Hkv][d]); q_all [batch][max_len][Hq][d]. Returns out (same
+        layout as q_all; rows past a sequence's length are left as they are)."""
+        for t in (k_all, v_all, q_all):
+            assert t.is_contiguous() and t.dtype == self.cfg.torch_dtype
+        max_len = int(q_all.shape[1])
+        need = _lib.spla_block_causal_workspace_size(self.params, self.batch, max_len)
+        if self._bc_ws is None or self._bc_ws.numel() < need:
+            self._bc_ws = torch.empty((need + 255) // 256 * 256, dtype=torch.uint8,
+                                      device=self.device)
+        if out is None:
+            out = torch.zeros_like(q_all)
+        ptr = lambda t: 0 if t is None else t.data_ptr()
+        _lib.spla_block_causal_forward(self.params, self.c, k_all.data_ptr(), v_all.data_ptr(),
+                                       q_all.data_ptr(), max_len, ptr(gamma), out.data_ptr(),
+                                       ptr(o_sparse), ptr(o_rla), self._bc_ws.data_ptr(),
+                                       self._bc_ws.numel(), self.dev_status.data_ptr(),
+                                       self._stream(stream))
+        return out
 
     def bulk_supported(self) -> bool:
         """Whether spla_append_kv_bulk takes this cache's shape (bf16, head_dim 128)."""

@@ -36,6 +36,7 @@ SPLA_WS_STAMP_BYTES = 16384
 EXPORTS = ("spla_cache_init", "spla_append_kv", "spla_append_kv_bulk",
            "spla_append_bulk_workspace_size", "spla_decode_workspace_size", "spla_decode",
            "spla_shard_candidates", "spla_shard_partials", "spla_shard_merge",
+           "spla_block_causal_workspace_size", "spla_block_causal_forward",
            "spla_decode_static_workspace", "spla_profile_events", "spla_profile_stamps",
            "spla_status_string", "spla_last_cuda_error", "spla_version")
 
@@ -90,13 +91,18 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.spla_shard_candidates.argtypes = [P, C, i32, vp, vp, vp, vp, sz, vp, vp]
     lib.spla_shard_partials.argtypes = [P, C, i32, vp, vp, vp, i32, vp, vp, sz, vp, vp]
     lib.spla_shard_merge.argtypes = [P, i32, vp, i32, vp, vp, vp, vp, vp, vp]
+    lib.spla_block_causal_workspace_size.argtypes = [P, i32, i32, ctypes.POINTER(sz)]
+    lib.spla_block_causal_forward.argtypes = [P, C, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp,
+                                              vp]
     lib.spla_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     lib.spla_profile_stamps.argtypes = [i32]
     for f in ("spla_cache_init", "spla_append_kv", "spla_append_kv_bulk",
               "spla_append_bulk_workspace_size", "spla_decode_workspace_size", "spla_decode",
            "spla_shard_candidates", "spla_shard_partials", "spla_shard_merge",
+           "spla_block_causal_workspace_size", "spla_block_causal_forward",
               "spla_decode_static_workspace", "spla_profile_events", "spla_profile_stamps",
-              "spla_shard_candidates", "spla_shard_partials", "spla_shard_merge"):
+              "spla_shard_candidates", "spla_shard_partials", "spla_shard_merge",
+              "spla_block_causal_workspace_size", "spla_block_causal_forward"):
         getattr(lib, f).restype = ctypes.c_int
     lib.spla_status_string.argtypes = [ctypes.c_int]
     lib.spla_status_string.restype = ctypes.c_char_p
@@ -160,6 +166,22 @@ def spla_shard_merge(params, batch, part_all, nshards, gamma, out, o_sparse, o_r
     _check("spla_shard_merge",
            load().spla_shard_merge(ctypes.byref(params), batch, part_all, nshards, gamma, out,
                                    o_sparse, o_rla, dev_status, stream))
+
+
+def spla_block_causal_workspace_size(params, batch, max_len) -> int:
+    n = ctypes.c_size_t(0)
+    _check("spla_block_causal_workspace_size",
+           load().spla_block_causal_workspace_size(ctypes.byref(params), batch, max_len,
+                                                   ctypes.byref(n)))
+    return n.value
+
+
+def spla_block_causal_forward(params, cache, k_all, v_all, q_all, max_len, gamma, out, o_sparse,
+                              o_rla, workspace, workspace_bytes, dev_status, stream=0):
+    _check("spla_block_causal_forward",
+           load().spla_block_causal_forward(ctypes.byref(params), ctypes.byref(cache), k_all,
+                                            v_all, q_all, max_len, gamma, out, o_sparse, o_rla,
+                                            workspace, workspace_bytes, dev_status, stream))
 
 
 def spla_decode_workspace_size(params, batch, max_blocks_per_seq) -> int:

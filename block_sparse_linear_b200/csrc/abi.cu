@@ -16,6 +16,15 @@ cudaError_t launch_append_bulk(const CacheView& c, const CUtensorMap& tk, const 
                                int32_t max_new, float* part, int32_t* status, cudaStream_t s);
 size_t bulk_workspace_bytes(int batch, int hkv, int d, int max_new);
 int shard_max_gathered();
+int bc_max_blocks();
+int bc_max_top_k();
+size_t bc_workspace_bytes(int batch, int hkv, int bs, int max_len);
+cudaError_t launch_block_causal_entry(const CacheView& c, const CUtensorMap& tk,
+                                      const CUtensorMap& tv, const void* k_all, int32_t max_len,
+                                      const void* q_all, const float* gamma, void* out,
+                                      float* o_sp, float* o_rl, int top_k, int n_sink,
+                                      int first_order, int no_rla, double scale, float eps,
+                                      char* ws, int32_t* status, cudaStream_t s);
 cudaError_t launch_shard_cand(const CacheView& c, const float* scores, int ld,
                               const uint32_t* bits, int nw, int top_k, int n_sink, int n_local,
                               int32_t first_block, const int32_t* global_nb, void* cand,
@@ -564,6 +573,65 @@ spla_status spla_shard_merge(const spla_params* params, int32_t batch, const dou
                                        params->head_dim, params->dtype, part_all, nshards, no_rla,
                                        eps, rms_gamma, out, o_sparse_dbg, o_rla_dbg, dev_status,
                                        (cudaStream_t)stream);
+    return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
+}
+
+
+// ------------------------------------------------------------------ block-causal form
+static spla_status check_block_causal(const spla_params* params, int32_t batch, int32_t max_len) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if (params->dtype != SPLA_BF16 || params->head_dim != 128 ||
+        params->num_q_heads / params->num_kv_heads > 4)
+        return SPLA_ERR_UNSUPPORTED;
+    if (batch <= 0 || max_len <= 0) return SPLA_ERR_INVALID_ARG;
+    if ((max_len + params->block_size - 1) / params->block_size > bc_max_blocks() ||
+        params->top_k > bc_max_top_k() || (int64_t)batch * max_len > INT32_MAX)
+        return SPLA_ERR_CAPACITY;
+    return SPLA_OK;
+}
+
+spla_status spla_block_causal_workspace_size(const spla_params* params, int32_t batch,
+                                             int32_t max_len, size_t* bytes) {
+    spla_status st = check_block_causal(params, batch, max_len);
+    if (st != SPLA_OK) return st;
+    if (!bytes) return SPLA_ERR_INVALID_ARG;
+    *bytes = bc_workspace_bytes(batch, params->num_kv_heads, params->block_size, max_len);
+    return SPLA_OK;
+}
+
+spla_status spla_block_causal_forward(const spla_params* params, const spla_cache* cache,
+                                      const void* k_all, const void* v_all, const void* q_all,
+                                      int32_t max_len, const float* rms_gamma, void* out,
+                                      float* o_sparse_dbg, float* o_rla_dbg, void* workspace,
+                                      size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    spla_status st = check_params(params);
+    if (st != SPLA_OK) return st;
+    if ((st = check_cache(cache)) != SPLA_OK) return st;
+    if ((st = check_block_causal(params, cache->batch, max_len)) != SPLA_OK) return st;
+    if (!k_all || !v_all || !q_all || !out) return SPLA_ERR_INVALID_ARG;
+    auto misaligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) != 0; };
+    if (misaligned(k_all) || misaligned(v_all) || misaligned(q_all) || !cache_aligned(cache) ||
+        misaligned(cache->blk_stats) || misaligned(cache->m))
+        return SPLA_ERR_INVALID_ARG;
+    if ((max_len + params->block_size - 1) / params->block_size > cache->max_blocks_per_seq)
+        return SPLA_ERR_CAPACITY;
+    const size_t need = bc_workspace_bytes(cache->batch, params->num_kv_heads, params->block_size,
+                                           max_len);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return SPLA_ERR_WORKSPACE;
+    const CacheView v = view_of(params, cache);
+    CUtensorMap tk, tv;
+    if (!make_input_map(&tk, k_all, v, max_len) || !make_input_map(&tv, v_all, v, max_len))
+        return SPLA_ERR_UNSUPPORTED;
+    const double scale = params->softmax_scale > 0.f ? (double)params->softmax_scale
+                                                     : 1.0 / sqrt((double)params->head_dim);
+    const float eps = params->rms_eps > 0.f ? params->rms_eps : 1e-6f;
+    cudaError_t e = launch_block_causal_entry(
+        v, tk, tv, k_all, max_len, q_all, rms_gamma, out, o_sparse_dbg, o_rla_dbg, params->top_k,
+        params->n_sink, (params->flags & SPLA_FLAG_FIRST_ORDER) ? 1 : 0,
+        (params->flags & SPLA_FLAG_NO_RLA) ? 1 : 0, scale, eps, static_cast<char*>(workspace),
+        dev_status, (cudaStream_t)stream);
     return e == cudaSuccess ? SPLA_OK : cuda_fail(e);
 }
 

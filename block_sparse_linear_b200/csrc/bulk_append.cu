@@ -454,6 +454,22 @@ cudaError_t launch_append_blocks(const CacheView& c, int dtype, const void* k_ne
 cudaError_t launch_append_advance(const CacheView& c, const int32_t* n_new, int32_t max_new,
                                   cudaStream_t s);
 
+// Partial states of a whole sequence block by block (one split per block of B
+// tokens): record (bh, j) holds S_j, z_j and m_j of block j's tokens. The inputs
+// are the sequences' tokens from position 0.
+cudaError_t launch_block_states(const CacheView& c, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const void* k_all, const int32_t* lens, int32_t max_len,
+                                float* rec, int32_t* status, cudaStream_t s) {
+    const int splits = (max_len + c.bs - 1) / c.bs;
+    cudaError_t e = cudaFuncSetAttribute(bulk_state_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kBulkSmem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(bulk_state_kernel, dim3(splits, c.batch * c.hkv), dim3(kBulkThreads),
+                      kBulkSmem, s, tk, tv, (const __nv_bfloat16*)k_all, lens, max_len, c.hkv,
+                      c.bs, rec, status);
+}
+
 // Order on the stream: state kernel (waits for everything before it, then lets the
 // next launch in), block kernel (runs beside it on the SMs' remaining shared memory
 // and registers; waits for the state kernel only at its end), merge, length advance.

@@ -281,6 +281,37 @@ SPLA_API spla_status spla_shard_merge(const spla_params* params, int32_t batch,
                              int32_t* dev_status, void* stream);
 
 /*
+ * The block-causal form over whole sequences (a prefill or training forward):
+ * query t of sequence b sees its tokens 0..t. Its own block J = t / B is
+ * attended exactly and causally; the complete earlier blocks 0..J-1 are scored
+ * (section 2.1) and the sink blocks plus the top_k of the rest attended exactly
+ * (ties to the lower block); the earlier blocks left out are covered by linear
+ * attention by subtraction (section 2.2) from the state of the tokens before
+ * block J; out = o_sparse + gamma * RMSNorm(o_rla) (section 2.3).
+ *   cache       : holds exactly each sequence's tokens 0..context_lens[b]-1,
+ *                 appended from k_all / v_all (its statistics, pools and final m
+ *                 are used; n_local is ignored: the query's own block plays it).
+ *   k_all, v_all: [batch][max_len][Hkv][d] bf16, the same tokens; q_all
+ *                 [batch][max_len][Hq][d] bf16; all 16-byte aligned.
+ *   out         : [batch][max_len][Hq][d] bf16; rows t >= context_lens[b] are not
+ *                 written. o_sparse_dbg, o_rla_dbg: the same layout in fp32, or NULL.
+ *   workspace   : spla_block_causal_workspace_size bytes, 256-byte aligned: per
+ *                 block states and the prefix states at every block boundary.
+ * Supported: bf16, head_dim 128, at most 4096 blocks per sequence, top_k <= 256
+ * (SPLA_ERR_UNSUPPORTED / SPLA_ERR_CAPACITY otherwise). Device faults as for
+ * spla_decode (a residual the fp32 sums cannot resolve sets
+ * SPLA_DEV_RLA_UNRESOLVED and gives o_rla = 0 for that query and head).
+ */
+SPLA_API spla_status spla_block_causal_workspace_size(const spla_params* params, int32_t batch,
+                                             int32_t max_len, size_t* bytes);
+
+SPLA_API spla_status spla_block_causal_forward(const spla_params* params, const spla_cache* cache,
+                                      const void* k_all, const void* v_all, const void* q_all,
+                                      int32_t max_len, const float* rms_gamma, void* out,
+                                      float* o_sparse_dbg, float* o_rla_dbg, void* workspace,
+                                      size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * Bytes of the library-owned scratch that spla_decode_static_workspace uses
  * on each device (one file-scope __device__ array, 256-byte aligned).
  */

@@ -234,3 +234,29 @@ def test_sharded_decode_host_checks(lib):
                                 None) == _lib.SPLA_ERR_INVALID_ARG
     assert lib.spla_shard_merge(B(p), 0, FAKE, 2, None, FAKE, None, None, None,
                                 None) == _lib.SPLA_ERR_INVALID_ARG
+
+
+def test_block_causal_forward_host_checks(lib):
+    """spla_block_causal_forward: bf16 / head_dim 128 / groups of at most 4 heads only, a
+    bounded block count and top_k, aligned inputs and a large enough workspace."""
+    B = ctypes.byref
+    p = _params()
+    c = _cache()
+    need = _lib.spla_block_causal_workspace_size(p, 4, 8192)
+    assert need == _lib.spla_block_causal_workspace_size(p, 4, 8192) > 0
+
+    def fwd(pp=p, k=FAKE, q=FAKE, max_len=8192, ws=FAKE, n=None):
+        return lib.spla_block_causal_forward(B(pp), B(c), k, FAKE, q, max_len, None, FAKE, None,
+                                             None, ws, need if n is None else n, None, None)
+
+    for bad in (_params(dtype=_lib.SPLA_F32), _params(head_dim=64, num_q_heads=8, num_kv_heads=2),
+                _params(num_q_heads=32, num_kv_heads=4)):
+        assert fwd(pp=bad) == _lib.SPLA_ERR_UNSUPPORTED
+    assert fwd(pp=_params(top_k=257)) == _lib.SPLA_ERR_CAPACITY
+    assert fwd(max_len=64 * 4096 + 1) == _lib.SPLA_ERR_CAPACITY
+    assert fwd(max_len=0) == _lib.SPLA_ERR_INVALID_ARG
+    assert fwd(k=None) == _lib.SPLA_ERR_INVALID_ARG
+    assert fwd(q=FAKE + 2) == _lib.SPLA_ERR_INVALID_ARG
+    assert fwd(ws=None) == _lib.SPLA_ERR_WORKSPACE
+    assert fwd(n=need - 1) == _lib.SPLA_ERR_WORKSPACE
+    assert fwd(ws=FAKE + 16) == _lib.SPLA_ERR_WORKSPACE
