@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--shards", type=int, default=0,
                     help="also time the context-sharded decode with the workload's sequences "
                          "split into this many shard caches on this GPU")
+    ap.add_argument("--no-block-causal", action="store_true",
+                    help="skip the block-causal forward measurement")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the bulk-append (prefill chunk) measurement")
     ap.add_argument("--also", default="cfg4",
@@ -375,6 +377,7 @@ def run_ours(args):
 
     prefill = measure_prefill("cfg4", dev, stream, flush) if not args.no_prefill else None
     sharded = measure_sharded(w, args.shards, K, W, dev, stream, flush) if args.shards > 0 else None
+    bcausal = measure_block_causal(dev, stream, flush) if not args.no_block_causal else None
 
     # ---- max over ranks (the same single collective on every rank)
     t_max, e2e_ms, tx_max = max_over_ranks(
@@ -421,6 +424,8 @@ def run_ours(args):
                 "clocks": mx["clocks"]}
         if sharded:
             res["sharded_emulation"] = sharded
+        if bcausal:
+            res["block_causal"] = bcausal
         if prefill:
             hbm_p = hbm
             prefill["bulk"]["frac_of_measured_peak" if peak_kind == "measured"
@@ -579,6 +584,71 @@ def measure_sharded(w, nshards, K, W, dev, stream, flush):
     del shards
     torch.cuda.empty_cache()
     return res
+
+
+def measure_block_causal(dev, stream, flush, n_tok=8192, K=5, W=3, loop_positions=256):
+    """The block-causal forward of one n_tok-token sequence with the 128K workload's heads
+    (32 q / 8 kv, d 128, block 64, top-k 32, bf16): spla_block_causal_forward on a cache
+    that holds the sequence (CUDA events, L2 flushed before each run), and, for
+    comparison, the same outputs as one-token appends and decodes with a local block,
+    timed over the sequence's last loop_positions positions and scaled to tokens/s."""
+    import torch
+    from block_sparse_linear_b200 import SplaConfig, SplaDecodeCache
+    hq, hkv, d, bs, k = 32, 8, 128, 64, 32
+    nb = -(-n_tok // bs)
+    g = torch.Generator(device=dev).manual_seed(9)
+    rnd = lambda *shape: torch.randn(shape, device=dev, generator=g).to(torch.bfloat16)
+    kk, vv, qq = rnd(1, n_tok, hkv, d), rnd(1, n_tok, hkv, d), rnd(1, n_tok, hq, d)
+    cfg = SplaConfig(num_q_heads=hq, num_kv_heads=hkv, head_dim=d, block_size=bs, top_k=k)
+    table = torch.arange(nb, dtype=torch.int32).reshape(1, nb)
+    cache = SplaDecodeCache(cfg, 1, table, nb, device=dev)
+    cache.append(kk, vv)
+    out = torch.empty_like(qq)
+    ts = []
+    for i in range(W + K):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.block_causal_forward(kk, vv, qq, None, out)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= W:
+            ts.append(e0.elapsed_time(e1))
+    ms = float(np.median(ts))
+    status = cache.status()
+    del cache
+    # the per-position path: one-token append + decode with the current block as local block
+    cfgl = SplaConfig(num_q_heads=hq, num_kv_heads=hkv, head_dim=d, block_size=bs, top_k=k,
+                      n_local=1)
+    cl = SplaDecodeCache(cfgl, 1, table, nb, device=dev)
+    o1 = torch.empty((1, hq, d), dtype=torch.bfloat16, device=dev)
+    n0 = n_tok - loop_positions - W                  # the last positions: the longest contexts
+    cl.append(kk[:, :n0].contiguous(), vv[:, :n0].contiguous())
+    for t in range(n0, n0 + W):
+        cl.append(kk[:, t:t + 1].contiguous(), vv[:, t:t + 1].contiguous())
+        cl.decode(qq[:, t].contiguous(), None, o1)
+    steps = [(kk[:, t:t + 1].contiguous(), vv[:, t:t + 1].contiguous(), qq[:, t].contiguous())
+             for t in range(n0 + W, n_tok)]
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for kt, vt, qt in steps:
+        cl.append(kt, vt)
+        cl.decode(qt, None, o1)
+    e1.record(stream)
+    e1.synchronize()
+    loop_ms = e0.elapsed_time(e1) / loop_positions
+    del cl
+    torch.cuda.empty_cache()
+    return {"workload": f"block-causal forward of one {n_tok}-token sequence, {hq} q / {hkv} kv "
+                        f"heads, d {d}, block {bs}, top-k {k}, bf16",
+            "runs": K, "warmup": W, "l2": "flushed before every run",
+            "ms_per_sequence": round(ms, 4), "tokens_per_s": round(n_tok / (ms * 1e-3), 1),
+            "dev_status": status,
+            "per_position_loop": {"positions_timed": loop_positions,
+                                  "ms_per_position": round(loop_ms, 5),
+                                  "tokens_per_s": round(1.0 / (loop_ms * 1e-3), 1)},
+            "speedup": round(loop_ms * n_tok / ms, 1)}
 
 
 def e2e_pass(w, cache, steps, s0, K, gamma, flush, dev, stream, ones):
