@@ -18,7 +18,9 @@
 //   bc_phi_kernel      phi = exp(k - m*) of every token, once (the kept tokens'
 //                      linear-attention weights become dot products with it);
 //   bc_query_kernel    grid (max_len, batch*Hkv), one warp per query head of the
-//                      group: fp64 block scores over the complete earlier blocks,
+//                      group, lanes over dimensions (every statistics, K, V and
+//                      phi row one coalesced load, dot products as warp sums):
+//                      fp64 block scores over the complete earlier blocks,
 //                      the head's top_k by repeated warp arg-max over (score,
 //                      lower block), exact online softmax over the kept blocks
 //                      and the causal part of block J (K/V from the paged pool),
