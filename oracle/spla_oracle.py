@@ -46,7 +46,10 @@ Readings where the pages leave a step open (the CUDA path makes the same ones):
     (first) and local (last) blocks are kept on top of the top-k only when a
     workload names them; when k or fewer candidates remain every block is kept;
  9. decode attends over the whole cache, the token just appended included;
-    an empty cache gives out = 0.
+    an empty cache gives out = 0;
+10. block-causal form: query t sees tokens 0..t, its own block exactly and
+    causally, the complete earlier blocks as candidates (top_k after any sink
+    blocks kept), the candidates left out by linear attention.
 """
 from __future__ import annotations
 
