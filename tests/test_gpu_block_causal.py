@@ -2,7 +2,7 @@
 oracle's block_causal_forward, every query position of every head.
 
 Sequences of ragged lengths (partial last blocks), two KV groups, with and without a
-sink block, and the first-order score flag. o_sparse is compared everywhere; o_rla
+sink block, the first-order score flag and the residual switched off. o_sparse is compared everywhere; o_rla
 and out where the residual's subtraction is well conditioned (kappa as in
 tests/parity.py, computed here from the tokens directly), and the count of
 ill-conditioned positions is asserted to be zero for these value distributions.
@@ -43,14 +43,15 @@ def _kappa(q, K, V, kept_tokens, J):
     return float(max(Dt / dr, np.abs(Nt).max() / nr))
 
 
-@pytest.mark.parametrize("n_sink,first_order", [(0, False), (1, False), (0, True)])
-def test_block_causal_forward_matches_oracle(n_sink, first_order):
-    rng = np.random.default_rng(17 + n_sink + 2 * first_order)
+@pytest.mark.parametrize("n_sink,first_order,no_rla",
+                         [(0, False, False), (1, False, False), (0, True, False), (1, False, True)])
+def test_block_causal_forward_matches_oracle(n_sink, first_order, no_rla):
+    rng = np.random.default_rng(17 + n_sink + 2 * first_order + 4 * no_rla)
     lens, hkv, G, top_k = (330, 200), 2, 4, 2
     batch, hq, max_len = len(lens), hkv * G, max(lens)
     nb = -(-max_len // BS)
     cfg = SplaConfig(num_q_heads=hq, num_kv_heads=hkv, head_dim=D, block_size=BS, top_k=top_k,
-                     n_sink=n_sink, first_order=first_order)
+                     n_sink=n_sink, first_order=first_order, no_rla=no_rla)
     to16 = lambda a: torch.from_numpy(a).to(torch.bfloat16)
     off = np.repeat(rng.normal(0.0, 0.5, (batch, nb, hkv, D)), BS, axis=1)[:, :max_len]
     K = to16(rng.standard_normal((batch, max_len, hkv, D)) + off)
@@ -71,7 +72,7 @@ def test_block_causal_forward_matches_oracle(n_sink, first_order):
     out, osp, orl = out.float().cpu().numpy(), osp.cpu().numpy(), orl.cpu().numpy()
     K64, V64, Q64 = K.double().numpy(), V.double().numpy(), Q.double().numpy()
     p = so.OracleParams(num_q_heads=hq, num_kv_heads=hkv, head_dim=D, block_size=BS,
-                        top_k=top_k, n_sink=n_sink, first_order=first_order)
+                        top_k=top_k, n_sink=n_sink, first_order=first_order, no_rla=no_rla)
     tol = parity.TOL["bf16"]
     ill = 0
     for b, L in enumerate(lens):
@@ -96,3 +97,5 @@ def test_block_causal_forward_matches_oracle(n_sink, first_order):
         # rows past the sequence's length are not written
         assert np.all(out[b, L:] == 0)
     assert ill == 0, ill
+    if no_rla:
+        assert np.all(orl == 0)
