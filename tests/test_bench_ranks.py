@@ -35,7 +35,7 @@ def _rank_main(rank, world, port, out):
 
 def test_max_over_ranks_gloo_world_2():
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
         got = dict(out)
@@ -101,7 +101,7 @@ def test_sharded_decode_gather_orders_shards_by_rank_gloo_world_2():
     """The all-gather between the sharded decode's phases stacks every rank's shards in
     global shard order (rank-major), as spla_shard_partials and spla_shard_merge expect."""
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_gather_main, args=(2, port, out), nprocs=2, join=True)
         got = dict(out)
