@@ -251,8 +251,9 @@ SPLA_API spla_status spla_decode(const spla_params* params, const spla_cache* ca
  *    sequence's top_k-th candidate, decodes them and writes one record per
  *    (sequence, query head): part [batch][Hq][SPLA_SHARD_REC(d)] fp64.
  * 4. The caller gathers every shard's part into part_all [nshards][batch][Hq][...].
- * 5. spla_shard_merge: out (and the debug outputs) exactly as spla_decode
- *    defines them, from part_all; any stream, no cache needed.
+ * 5. spla_shard_merge: out (and the debug outputs) as spla_decode defines them
+ *    (the same values up to the order of the fp32 sums), from part_all; any
+ *    stream, no cache needed.
  * The workspace is spla_decode_workspace_size(params, batch, max_blocks_per_seq)
  * bytes. Argument checks and device faults as for spla_decode;
  * SPLA_ERR_CAPACITY when nshards * top_k exceeds 4096.
